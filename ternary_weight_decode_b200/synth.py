@@ -1,0 +1,124 @@
+"""Seeded synthetic inputs for the ternary weight path.
+
+This module holds input generation only: no packing, quantisation or
+dot-product arithmetic lives here.  Both the CUDA path and the CPU oracle
+consume what it produces.
+
+Weights and scales come from a counter-based generator so that any single
+row can be regenerated on its own, on the host or on the device:
+
+* ``mix64`` is the SplitMix64 output function (Steele, Lea & Flood,
+  "Fast splittable pseudorandom number generators", OOPSLA 2014; the
+  public-domain reference code by S. Vigna).
+* ``h(seed, stream, idx)`` is the ``idx``-th output (0-based) of SplitMix64
+  whose state starts at ``key = mix64(seed * GAMMA + stream)``, i.e.
+  ``mix64(key + (idx + 1) * GAMMA)`` modulo 2**64.
+
+A trit is drawn from ``u = h >> 32``: -1 when ``u < T_NEG``, +1 when
+``u >= T_POS``, else 0 (P(-1) = P(+1) = 0.3, P(0) = 0.4, the distribution
+of the single-GEMV workload).  A group scale is drawn from ``u24 = h >> 40``
+as ``fp16(fp32(fp32(u24 * 2**-24) * 0.045) + 0.005)`` with every fp32 step
+rounded to nearest, giving scales in [0.005, 0.05).
+
+The device generator in ``csrc/synth.cu`` implements the same definition;
+a GPU test checks the two bit for bit.
+
+Activations are drawn on the host with numpy's PCG64: N(0, 1), 1% of the
+entries (``rng.random() < 0.01``) multiplied by 20, stored as fp16.
+"""
+from __future__ import annotations
+
+import numpy as np
+
+GAMMA = 0x9E3779B97F4A7C15
+MASK64 = (1 << 64) - 1
+T_NEG = 1288490189  # ceil(0.3 * 2**32)
+T_POS = 3006477108  # ceil(0.7 * 2**32)
+
+# Stream ids: projection p of layer l uses streams STREAM_BASE(l, p) (trits)
+# and STREAM_BASE(l, p) + 1 (scales).
+PROJ_QKV, PROJ_O, PROJ_GATE, PROJ_UP, PROJ_DOWN = 0, 1, 2, 3, 4
+
+
+def stream_id(layer: int, proj: int, scales: bool = False) -> int:
+    return (layer * 16 + proj * 2 + (1 if scales else 0)) & MASK64
+
+
+def mix64_int(z: int) -> int:
+    """SplitMix64 output function on a Python int (mod 2**64)."""
+    z &= MASK64
+    z = ((z ^ (z >> 30)) * 0xBF58476D1CE4E5B9) & MASK64
+    z = ((z ^ (z >> 27)) * 0x94D049BB133111EB) & MASK64
+    return z ^ (z >> 31)
+
+
+def stream_key(seed: int, stream: int) -> int:
+    return mix64_int(((seed * GAMMA) + stream) & MASK64)
+
+
+def _mix64_np(z: np.ndarray) -> np.ndarray:
+    z = z.astype(np.uint64, copy=True)
+    z ^= z >> np.uint64(30)
+    z *= np.uint64(0xBF58476D1CE4E5B9)
+    z ^= z >> np.uint64(27)
+    z *= np.uint64(0x94D049BB133111EB)
+    z ^= z >> np.uint64(31)
+    return z
+
+
+def hash_at(seed: int, stream: int, idx: np.ndarray) -> np.ndarray:
+    """h(seed, stream, idx) for an array of uint64 counters."""
+    key = np.uint64(stream_key(seed, stream))
+    idx = np.asarray(idx, dtype=np.uint64)
+    with np.errstate(over="ignore"):
+        x = key + (idx + np.uint64(1)) * np.uint64(GAMMA)
+    return _mix64_np(x)
+
+
+def trits_rows(seed: int, stream: int, rows: np.ndarray, K: int) -> np.ndarray:
+    """Trits int8 [len(rows), K] of the matrix (seed, stream) at the given rows."""
+    rows = np.asarray(rows, dtype=np.uint64).reshape(-1, 1)
+    idx = rows * np.uint64(K) + np.arange(K, dtype=np.uint64).reshape(1, -1)
+    u = hash_at(seed, stream, idx) >> np.uint64(32)
+    out = np.zeros(u.shape, dtype=np.int8)
+    out[u < np.uint64(T_NEG)] = -1
+    out[u >= np.uint64(T_POS)] = 1
+    return out
+
+
+def trits(seed: int, stream: int, N: int, K: int) -> np.ndarray:
+    """Trits int8 [N, K] in {-1, 0, +1}."""
+    return trits_rows(seed, stream, np.arange(N), K)
+
+
+def scales_rows(seed: int, stream: int, rows: np.ndarray, G: int) -> np.ndarray:
+    """fp16 group scales [len(rows), G] as numpy float16."""
+    rows = np.asarray(rows, dtype=np.uint64).reshape(-1, 1)
+    idx = rows * np.uint64(G) + np.arange(G, dtype=np.uint64).reshape(1, -1)
+    u24 = (hash_at(seed, stream, idx) >> np.uint64(40)).astype(np.float32)
+    a = u24 * np.float32(2.0 ** -24)  # exact: u24 < 2**24
+    b = a * np.float32(0.045)
+    c = b + np.float32(0.005)
+    return c.astype(np.float16)
+
+
+def scales(seed: int, stream: int, N: int, G: int) -> np.ndarray:
+    return scales_rows(seed, stream, np.arange(N), G)
+
+
+def activations(seed: int, M: int, K: int) -> np.ndarray:
+    """fp16 activations [M, K]: N(0,1) with 1% of entries scaled by 20."""
+    rng = np.random.default_rng(seed)
+    x = rng.standard_normal(M * K)
+    mask = rng.random(M * K) < 0.01
+    x[mask] *= 20.0
+    return x.astype(np.float16).reshape(M, K)
+
+
+def activation_rows(seeds, K: int) -> np.ndarray:
+    """One independently seeded fp16 row per seed (multi-slot decode rows)."""
+    return np.concatenate([activations(int(s), 1, K) for s in seeds], axis=0)
+
+
+def groups(K: int, group: int = 128) -> int:
+    return (K + group - 1) // group
