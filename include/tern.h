@@ -1,0 +1,206 @@
+/*
+ * tern.h -- C ABI of libtern.so, the B200 (sm_100a) ternary-weight path.
+ *
+ * What the library computes (the pages this method is described on):
+ *  - "Ternary Bonsai 2 27B: 8GB 显卡硬塞 27B 三元模型，能跑，但我大概率不会真用"
+ *    (171host.com), section "Decode 为什么只能算一般": batch-1 decode reads the
+ *    packed weights once per token; the kernel unpacks base-3 codes, restores
+ *    -1/0/+1, reads the group scale and takes an integer dot product with the
+ *    quantised activation, never writing dequantised weights back to memory;
+ *    gate/up + SwiGLU run as one fused kernel sharing the Hadamard-rotated,
+ *    quantised input; activations are re-quantised per token between matmuls.
+ *  - "三值权重 27B 压到 5.9GB｜本地部署成本账单重算" (blog.4sapi.com), section 三:
+ *    weights in {-1, 0, +1} with one FP16 scale per group; add/subtract by
+ *    sign, then multiply by the group scale.
+ *  - Same Bonsai page, section "后面还有没有优化空间": re-tile codes and scales
+ *    at load time into the order the integer dot product consumes them.
+ *
+ * Conventions for every call:
+ *  - Every pointer argument marked "device" is CUDA device memory owned by
+ *    the caller.  The library allocates nothing, frees nothing and never
+ *    synchronises the device; every call is asynchronous on `stream`
+ *    (a cudaStream_t; NULL = legacy default stream) and may be captured in a
+ *    CUDA graph.
+ *  - Arguments are validated on the host before any launch; a violation
+ *    returns TERN_EINVAL and launches nothing.  A failed launch returns
+ *    TERN_ECUDA; tern_last_error() then holds the CUDA message.  No call
+ *    aborts, throws or exits.  There is no CPU fallback.
+ *  - Compute kernels are launched with programmatic dependent launch: they
+ *    may begin before the previous kernel on the stream has finished, but
+ *    read activations and write outputs only after it has.
+ */
+#ifndef TERN_H
+#define TERN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    TERN_OK = 0,
+    TERN_EINVAL = 1,       /* bad argument (shape, alignment, pointer, format) */
+    TERN_ECUDA = 2,        /* a CUDA launch or query failed */
+    TERN_EUNSUPPORTED = 3, /* valid request this build does not implement */
+    TERN_ETIMEOUT = 4      /* a bounded device-side wait ran out */
+} tern_status;
+
+/* Weight formats.  Both hold one trit per weight, t = w + 1 in {0, 1, 2}. */
+typedef enum {
+    TERN_FMT_BASE3 = 0, /* 5 trits per byte (PTQ1_0-style), 1.6 bit/trit */
+    TERN_FMT_2BIT = 1   /* 4 trits per byte (PQ2-style), 2 bit/trit */
+} tern_format;
+
+/* Bit 0 of tern_matrix.flags: the packed codes and scales are not written by
+ * any work still pending on the stream, so a compute kernel may start
+ * streaming them before the previous kernel on the stream has finished. */
+#define TERN_MATRIX_STATIC 1
+
+/* act_quant_fwht flag: fold a weightless RMSNorm of the (unrotated) row into
+ * the scale, s_x *= fp32(1/sqrt(mean_k x_k^2 + 1e-6)); q is unchanged. */
+#define TERN_QUANT_RMSNORM 1
+
+/*
+ * A packed weight matrix W [N][K] in the device layout written by tern_pack
+ * or tern_import:
+ *   TERN_FMT_BASE3 (D3): 4-byte word w of a row covers K in [20w, 20w+20);
+ *     byte j of the word holds the trits at K = 20w + j + 4i, i = 0..4, as
+ *     y = ceil(256 V / 243) with V = sum_i t_i 3^(4-i).  Row bytes used:
+ *     4*ceil(K/20).
+ *   TERN_FMT_2BIT (D2): 4-byte word w covers K in [16w, 16w+16); bits
+ *     [2i, 2i+1] of byte j hold t for K = 16w + 4i + j.  Row bytes used:
+ *     4*ceil(K/16).
+ *   Positions past K hold t = 1 (w = 0); bytes past the used row bytes are 0.
+ * scales: fp16 bit patterns [N][ceil(K/group)], one per group of `group`
+ * consecutive K positions of a row (the last group may be partial).
+ */
+typedef struct tern_matrix {
+    int32_t fmt;           /* tern_format */
+    int32_t N;             /* output rows, >= 1 */
+    int32_t K;             /* input length, >= 1 */
+    int32_t group;         /* scale group along K; this build supports 128 */
+    int64_t row_stride;    /* bytes between rows of `packed`: a multiple of 16,
+                              >= the used row bytes */
+    const void *packed;    /* device, 16-byte aligned, N * row_stride bytes */
+    const uint16_t *scales;/* device, 2-byte aligned, N * ceil(K/group) fp16 */
+    int32_t flags;         /* TERN_MATRIX_STATIC or 0 */
+    int32_t reserved;      /* must be 0 */
+} tern_matrix;
+
+/* Human-readable name of a status code (static storage). */
+const char *tern_status_string(tern_status s);
+
+/* Message of the last failure on the calling host thread ("" if none). */
+const char *tern_last_error(void);
+
+/*
+ * Sizes of the device layout for an N x K matrix: the minimal row stride
+ * (used row bytes rounded up to 16), the packed bytes N*row_stride and the
+ * scale bytes 2*N*ceil(K/group).  Any output pointer may be NULL.
+ */
+tern_status tern_packed_size(int32_t fmt, int32_t N, int32_t K, int32_t group,
+                             int64_t *row_stride, size_t *packed_bytes,
+                             size_t *scale_bytes);
+
+/* Bytes per row of the canonical (file) encodings: base-3 = ceil(K/5)
+ * (byte value sum_{i<5} t_i 3^i over K = 5j+i, least significant digit
+ * first), 2-bit = ceil(K/4) (bits [2i,2i+1] of byte j hold K = 4j+i). */
+tern_status tern_canonical_row_bytes(int32_t fmt, int32_t K, int64_t *bytes);
+
+/*
+ * Pack trits into the device layout.
+ *  trits: device int8 [N][K] in {-1, 0, +1}.
+ *  packed_out: device, 16-byte aligned, N*row_stride bytes (row_stride as in
+ *    tern_matrix).  Every byte of every row is written.
+ *  d_invalid: optional device int32 counter (may be NULL); the number of
+ *    trits outside {-1,0,+1} is added to it (they are packed as 0).
+ */
+tern_status tern_pack(int32_t fmt, const int8_t *trits, int32_t N, int32_t K,
+                      void *packed_out, int64_t row_stride, int32_t *d_invalid,
+                      void *stream);
+
+/* Inverse of tern_pack: trits_out device int8 [N][K].  Invalid codes (D3
+ * bytes that are no code, D2 fields equal to 3, padding digits other than
+ * t = 1) are counted in d_invalid (may be NULL) and unpacked as 0. */
+tern_status tern_unpack(const tern_matrix *W, int8_t *trits_out,
+                        int32_t *d_invalid, void *stream);
+
+/* Load-time re-tile: canonical bytes (device [N][canonical row bytes],
+ * rows contiguous) into the device layout.  Invalid canonical codes are
+ * counted in d_invalid (may be NULL). */
+tern_status tern_import(int32_t fmt, const uint8_t *canonical, int32_t N,
+                        int32_t K, void *packed_out, int64_t row_stride,
+                        int32_t *d_invalid, void *stream);
+
+/* Device layout back to canonical bytes (device [N][canonical row bytes]). */
+tern_status tern_export(const tern_matrix *W, uint8_t *canonical_out,
+                        int32_t *d_invalid, void *stream);
+
+/*
+ * Per-token int8 activation quantisation with an optional 128-point
+ * Walsh-Hadamard rotation (Bonsai page, "Decode 为什么只能算一般": the FFN
+ * input is Hadamard-rotated once for gate and up; activations are quantised
+ * per token).  Row m of x (ldx elements apart, fp16 if x_is_fp16 else fp32):
+ *   x^ = x, or x^ = H x per 128-block (unnormalised Sylvester butterflies in
+ *        fp32, stages h = 1..64) when fwht_block == 128 (needs K % 128 == 0);
+ *   amax = max_k |x^_k|;  inv = 127/amax (IEEE fp32 division);
+ *   q[m][k] = clamp(rint_half_even(x^_k * inv), -127, 127) for k < K,
+ *   q[m][k] = 0 for K <= k < ldq;
+ *   s_x[m] = amax/127, times fp32(1/sqrt(128)) when rotated;
+ *   amax == 0 gives s_x = 0 and q = 0;
+ *   with TERN_QUANT_RMSNORM in flags, s_x is also divided by the row's rms.
+ *  x: device, 16-byte aligned, ldx a multiple of 8 (fp16) or 4 (fp32).
+ *  q: device int8 [M][ldq], 16-byte aligned, ldq >= K, ldq % 16 == 0.
+ *  s_x: device fp32 [M].  Inputs must be finite.
+ */
+tern_status act_quant_fwht(const void *x, int32_t x_is_fp16, int32_t M,
+                           int32_t K, int32_t ldx, int32_t fwht_block,
+                           int32_t flags, int8_t *q, int32_t ldq, float *s_x,
+                           void *stream);
+
+/*
+ * Ternary GEMV / skinny GEMM for decode, M = 1..16 token rows:
+ *   y[m][n] = residual[m][n] + s_x[m] * sum_g s_w[n][g] * P[m][n][g],
+ *   P[m][n][g] = sum_{k in group g} w[n][k] * q[m][k]   (exact int32),
+ * with residual taken as 0 when `residual` is NULL.
+ *  q: device int8 [M][ldq], 16-byte aligned, ldq >= K, ldq % 16 == 0
+ *     (bytes past K are ignored).  s_x: device fp32 [M].
+ *  residual, y: device fp32 [M][ldy], ldy >= N; residual may equal y.
+ */
+tern_status tern_gemv(const tern_matrix *W, const int8_t *q, int32_t ldq,
+                      const float *s_x, int32_t M, const float *residual,
+                      float *y, int32_t ldy, void *stream);
+
+/*
+ * Fused gate/up + SwiGLU (Bonsai page, "Decode 为什么只能算一般"):
+ *   g = Wg x^, u = Wu x^ (each as in tern_gemv, same q and s_x),
+ *   h[m][n] = g * sigmoid(g) * u,  sigmoid(z) = 1/(1+exp(-z)).
+ *  Wg and Wu must have the same fmt, N, K and group.  h: device fp32
+ *  [M][ldh], ldh >= N.
+ */
+tern_status tern_gateup_swiglu(const tern_matrix *Wg, const tern_matrix *Wu,
+                               const int8_t *q, int32_t ldq, const float *s_x,
+                               int32_t M, float *h, int32_t ldh, void *stream);
+
+/*
+ * Test hook: the exact integer group partials P[m][n][g] (device int32
+ * [M][N][ceil(K/group)]) of the same kernels tern_gemv runs.
+ */
+tern_status tern_debug_group_partials(const tern_matrix *W, const int8_t *q,
+                                      int32_t ldq, int32_t M, int32_t *P,
+                                      void *stream);
+
+/*
+ * Reads and clears the device error word of the current device: 0 when no
+ * bounded wait in a kernel ran out since the last call, else a nonzero code.
+ * Synchronises `stream`.
+ */
+tern_status tern_device_error(int32_t *code_out, void *stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* TERN_H */

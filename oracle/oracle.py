@@ -71,7 +71,7 @@ def _load():
             lib.oracle_d3_decode_value.restype = i32
             lib.oracle_d3_decode_value.argtypes = [i32]
             lib.oracle_act_quant.restype = i32
-            lib.oracle_act_quant.argtypes = [p, i64, i64, i32, p, p]
+            lib.oracle_act_quant.argtypes = [p, i64, i64, i32, i32, p, p]
             lib.oracle_fwht128_f32.restype = None
             lib.oracle_fwht128_f32.argtypes = [p]
             lib.oracle_fwht128_f64.restype = None
@@ -203,13 +203,14 @@ def fwht128_f64(v: np.ndarray) -> np.ndarray:
     return v
 
 
-def act_quant(x: np.ndarray, fwht_block: int = 0):
+def act_quant(x: np.ndarray, fwht_block: int = 0, rmsnorm: bool = False):
     """Returns (q int8 [M, K], s_x fp32 [M]) for fp16 or fp32 input x [M, K]."""
     x = _c(np.asarray(x).astype(np.float32), np.float32)
     M, K = x.shape
     q = np.zeros((M, K), np.int8)
     s = np.zeros((M,), np.float32)
-    _check(_load().oracle_act_quant(_ptr(x), M, K, fwht_block, _ptr(q), _ptr(s)), "act_quant")
+    _check(_load().oracle_act_quant(_ptr(x), M, K, fwht_block, 1 if rmsnorm else 0, _ptr(q),
+                                   _ptr(s)), "act_quant")
     return q, s
 
 

@@ -43,6 +43,9 @@
  *     h = 1, 2, ..., 64 with (a, b) -> (a + b, a - b); the orthonormal
  *     1/sqrt(128) is folded into s_x (s_x = fp32(fp32(amax/127) * fp32(1/sqrt(128)))).
  *  R8 SwiGLU: h = g * sigmoid(g) * u, sigmoid(z) = 1 / (1 + exp(-z)).
+ *  R9 decode chain glue (the pages give no norm or attention detail): a
+ *     weightless RMSNorm of the unrotated row folded into the scale only,
+ *     s_x / sqrt(mean(x^2) + 1e-6), which leaves every int8 code unchanged.
  *
  * Device layouts (the "load-time retile into consumption order" suggested on
  * [BONSAI], section "后面还有没有优化空间"):
@@ -295,13 +298,19 @@ void oracle_fwht128_f64(double *v) {
 /* x: fp32 [M][K] (fp16 inputs are passed as their exact fp32 values).
  * q: int8 [M][K]; s_x: fp32 [M]. */
 int oracle_act_quant(const float *x, int64_t M, int64_t K, int fwht_block,
-                     int8_t *q, float *s_x) {
+                     int rmsnorm, int8_t *q, float *s_x) {
     if (fwht_block != 0 && fwht_block != 128) return ORACLE_EINVAL;
     if (fwht_block == 128 && K % 128 != 0) return ORACLE_EINVAL;
     float *v = (float *)malloc((size_t)(K > 0 ? K : 1) * sizeof(float));
     if (!v) return ORACLE_EINVAL;
     for (int64_t m = 0; m < M; ++m) {
         memcpy(v, x + m * K, (size_t)K * sizeof(float));
+        double inv_rms = 1.0;
+        if (rmsnorm) {
+            double ss = 0.0;
+            for (int64_t k = 0; k < K; ++k) ss += (double)v[k] * (double)v[k];
+            inv_rms = 1.0 / sqrt(ss / (double)K + 1e-6);
+        }
         if (fwht_block == 128)
             for (int64_t b = 0; b < K / 128; ++b) oracle_fwht128_f32(v + 128 * b);
         float amax = 0.0f;
@@ -324,7 +333,7 @@ int oracle_act_quant(const float *x, int64_t M, int64_t K, int fwht_block,
         }
         volatile float s = amax / 127.0f;
         if (fwht_block == 128) s = s * INV_SQRT128_F;
-        s_x[m] = s;
+        s_x[m] = rmsnorm ? (float)((double)s * inv_rms) : s;
     }
     free(v);
     return ORACLE_OK;

@@ -1,0 +1,273 @@
+// tern_api.cu -- the extern "C" boundary of libtern (declared in tern.h):
+// argument validation on the host, then one launch per call on the caller's
+// stream.  No allocation, no synchronisation, no CPU fallback.
+#include <stdio.h>
+#include <string.h>
+
+#include "tern_common.cuh"
+#include "tern_internal.h"
+
+namespace {
+
+thread_local char g_last_error[512] = "";
+
+tern_status fail(tern_status s, const char *fmt, const char *detail = "") {
+    snprintf(g_last_error, sizeof(g_last_error), fmt, detail);
+    return s;
+}
+
+tern_status cuda_status(cudaError_t e, const char *what) {
+    if (e == cudaSuccess) return TERN_OK;
+    snprintf(g_last_error, sizeof(g_last_error), "%s: %s", what, cudaGetErrorString(e));
+    return TERN_ECUDA;
+}
+
+bool aligned(const void *p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+bool valid_fmt(int32_t fmt) { return fmt == TERN_FMT_BASE3 || fmt == TERN_FMT_2BIT; }
+
+tern_status check_matrix(const tern_matrix *W, const char *name) {
+    if (!W) return fail(TERN_EINVAL, "%s: null matrix", name);
+    if (!valid_fmt(W->fmt)) return fail(TERN_EINVAL, "%s: unknown format", name);
+    if (W->N < 1 || W->K < 1) return fail(TERN_EINVAL, "%s: N and K must be >= 1", name);
+    if (W->group != 128) return fail(TERN_EUNSUPPORTED, "%s: only group = 128 is supported", name);
+    if (W->row_stride % 16 != 0 || W->row_stride < tern::device_row_bytes(W->fmt, W->K))
+        return fail(TERN_EINVAL, "%s: row_stride must be a multiple of 16 and >= the used row bytes",
+                    name);
+    if (!W->packed || !aligned(W->packed, 16))
+        return fail(TERN_EINVAL, "%s: packed must be a 16-byte aligned device pointer", name);
+    if (!W->scales || !aligned(W->scales, 2))
+        return fail(TERN_EINVAL, "%s: scales must be a 2-byte aligned device pointer", name);
+    if (W->flags & ~TERN_MATRIX_STATIC) return fail(TERN_EINVAL, "%s: unknown flag bits", name);
+    if (W->reserved != 0) return fail(TERN_EINVAL, "%s: reserved must be 0", name);
+    return TERN_OK;
+}
+
+tern_status check_activations(const int8_t *q, int32_t ldq, int32_t K, const float *s_x,
+                              int32_t M) {
+    if (M < 1 || M > 16) return fail(TERN_EINVAL, "M must be in 1..16%s");
+    if (!q || !aligned(q, 16)) return fail(TERN_EINVAL, "q must be a 16-byte aligned device pointer%s");
+    if (ldq < K || ldq % 16 != 0) return fail(TERN_EINVAL, "ldq must be >= K and a multiple of 16%s");
+    if (!s_x || !aligned(s_x, 4)) return fail(TERN_EINVAL, "s_x must be a 4-byte aligned device pointer%s");
+    return TERN_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char *tern_status_string(tern_status s) {
+    switch (s) {
+        case TERN_OK: return "TERN_OK";
+        case TERN_EINVAL: return "TERN_EINVAL (invalid argument)";
+        case TERN_ECUDA: return "TERN_ECUDA (CUDA error)";
+        case TERN_EUNSUPPORTED: return "TERN_EUNSUPPORTED (not supported by this build)";
+        case TERN_ETIMEOUT: return "TERN_ETIMEOUT (bounded device wait ran out)";
+    }
+    return "unknown tern_status";
+}
+
+const char *tern_last_error(void) { return g_last_error; }
+
+tern_status tern_packed_size(int32_t fmt, int32_t N, int32_t K, int32_t group, int64_t *row_stride,
+                             size_t *packed_bytes, size_t *scale_bytes) {
+    if (!valid_fmt(fmt)) return fail(TERN_EINVAL, "unknown format%s");
+    if (N < 1 || K < 1 || group < 1) return fail(TERN_EINVAL, "N, K and group must be >= 1%s");
+    int64_t stride = (tern::device_row_bytes(fmt, K) + 15) / 16 * 16;
+    if (row_stride) *row_stride = stride;
+    if (packed_bytes) *packed_bytes = static_cast<size_t>(stride) * static_cast<size_t>(N);
+    if (scale_bytes)
+        *scale_bytes = 2u * static_cast<size_t>(N) * static_cast<size_t>(tern::ceil_div(K, group));
+    return TERN_OK;
+}
+
+tern_status tern_canonical_row_bytes(int32_t fmt, int32_t K, int64_t *bytes) {
+    if (!valid_fmt(fmt)) return fail(TERN_EINVAL, "unknown format%s");
+    if (K < 1 || !bytes) return fail(TERN_EINVAL, "K must be >= 1 and bytes non-null%s");
+    *bytes = tern::canonical_row_bytes(fmt, K);
+    return TERN_OK;
+}
+
+tern_status tern_pack(int32_t fmt, const int8_t *trits, int32_t N, int32_t K, void *packed_out,
+                      int64_t row_stride, int32_t *d_invalid, void *stream) {
+    if (!valid_fmt(fmt)) return fail(TERN_EINVAL, "tern_pack: unknown format%s");
+    if (N < 1 || K < 1) return fail(TERN_EINVAL, "tern_pack: N and K must be >= 1%s");
+    if (!trits || !packed_out || !aligned(packed_out, 16))
+        return fail(TERN_EINVAL, "tern_pack: null pointer or packed_out not 16-byte aligned%s");
+    if (row_stride % 16 != 0 || row_stride < tern::device_row_bytes(fmt, K))
+        return fail(TERN_EINVAL, "tern_pack: bad row_stride%s");
+    return cuda_status(tern::launch_pack(fmt, trits, N, K, packed_out, row_stride, d_invalid,
+                                         static_cast<cudaStream_t>(stream)),
+                       "tern_pack");
+}
+
+tern_status tern_unpack(const tern_matrix *W, int8_t *trits_out, int32_t *d_invalid, void *stream) {
+    tern_status st = check_matrix(W, "tern_unpack");
+    if (st != TERN_OK) return st;
+    if (!trits_out) return fail(TERN_EINVAL, "tern_unpack: null output%s");
+    return cuda_status(tern::launch_unpack(W->fmt, W->packed, W->N, W->K, W->row_stride, trits_out,
+                                           d_invalid, static_cast<cudaStream_t>(stream)),
+                       "tern_unpack");
+}
+
+tern_status tern_import(int32_t fmt, const uint8_t *canonical, int32_t N, int32_t K,
+                        void *packed_out, int64_t row_stride, int32_t *d_invalid, void *stream) {
+    if (!valid_fmt(fmt)) return fail(TERN_EINVAL, "tern_import: unknown format%s");
+    if (N < 1 || K < 1) return fail(TERN_EINVAL, "tern_import: N and K must be >= 1%s");
+    if (!canonical || !packed_out || !aligned(packed_out, 16))
+        return fail(TERN_EINVAL, "tern_import: null pointer or packed_out not 16-byte aligned%s");
+    if (row_stride % 16 != 0 || row_stride < tern::device_row_bytes(fmt, K))
+        return fail(TERN_EINVAL, "tern_import: bad row_stride%s");
+    return cuda_status(tern::launch_import(fmt, canonical, N, K, packed_out, row_stride, d_invalid,
+                                           static_cast<cudaStream_t>(stream)),
+                       "tern_import");
+}
+
+tern_status tern_export(const tern_matrix *W, uint8_t *canonical_out, int32_t *d_invalid,
+                        void *stream) {
+    tern_status st = check_matrix(W, "tern_export");
+    if (st != TERN_OK) return st;
+    if (!canonical_out) return fail(TERN_EINVAL, "tern_export: null output%s");
+    return cuda_status(tern::launch_export(W->fmt, W->packed, W->N, W->K, W->row_stride,
+                                           canonical_out, d_invalid,
+                                           static_cast<cudaStream_t>(stream)),
+                       "tern_export");
+}
+
+tern_status act_quant_fwht(const void *x, int32_t x_is_fp16, int32_t M, int32_t K, int32_t ldx,
+                           int32_t fwht_block, int32_t flags, int8_t *q, int32_t ldq, float *s_x,
+                           void *stream) {
+    if (M < 1 || K < 1) return fail(TERN_EINVAL, "act_quant_fwht: M and K must be >= 1%s");
+    if (K > 49152) return fail(TERN_EUNSUPPORTED, "act_quant_fwht: K > 49152 is not supported%s");
+    if (fwht_block != 0 && fwht_block != 128)
+        return fail(TERN_EINVAL, "act_quant_fwht: fwht_block must be 0 or 128%s");
+    if (flags & ~TERN_QUANT_RMSNORM) return fail(TERN_EINVAL, "act_quant_fwht: unknown flag bits%s");
+    if (fwht_block == 128 && K % 128 != 0)
+        return fail(TERN_EINVAL, "act_quant_fwht: the Hadamard rotation needs K %% 128 == 0%s");
+    if (!x || !aligned(x, 16)) return fail(TERN_EINVAL, "act_quant_fwht: x must be 16-byte aligned%s");
+    if (ldx < K || ldx % (x_is_fp16 ? 8 : 4) != 0)
+        return fail(TERN_EINVAL, "act_quant_fwht: ldx must be >= K and keep rows 16-byte aligned%s");
+    if (!q || !aligned(q, 16) || ldq < K || ldq % 16 != 0)
+        return fail(TERN_EINVAL, "act_quant_fwht: q must be 16-byte aligned with ldq >= K, ldq %% 16 == 0%s");
+    if (!s_x || !aligned(s_x, 4)) return fail(TERN_EINVAL, "act_quant_fwht: bad s_x%s");
+    return cuda_status(tern::launch_act_quant(x, x_is_fp16 != 0, M, K, ldx, fwht_block, flags, q, ldq, s_x,
+                                              static_cast<cudaStream_t>(stream)),
+                       "act_quant_fwht");
+}
+
+static tern_status run_gemv(tern::GemvLaunch &L, const char *name, cudaStream_t s) {
+    const char *why = nullptr;
+    cudaError_t e = tern::launch_gemv(L, s, &why);
+    if (why) return fail(TERN_EUNSUPPORTED, "%s", why);
+    return cuda_status(e, name);
+}
+
+tern_status tern_gemv(const tern_matrix *W, const int8_t *q, int32_t ldq, const float *s_x,
+                      int32_t M, const float *residual, float *y, int32_t ldy, void *stream) {
+    tern_status st = check_matrix(W, "tern_gemv");
+    if (st != TERN_OK) return st;
+    st = check_activations(q, ldq, W->K, s_x, M);
+    if (st != TERN_OK) return st;
+    if (!y || !aligned(y, 4) || ldy < W->N) return fail(TERN_EINVAL, "tern_gemv: bad y or ldy%s");
+    if (residual && !aligned(residual, 4)) return fail(TERN_EINVAL, "tern_gemv: bad residual%s");
+    tern::GemvLaunch L = {};
+    L.mode = tern::kModeGemv;
+    L.fmt = W->fmt;
+    L.N = W->N;
+    L.K = W->K;
+    L.G = static_cast<int>(tern::ceil_div(W->K, W->group));
+    L.row_bytes = tern::device_row_bytes(W->fmt, W->K);
+    L.row_stride = W->row_stride;
+    L.packed[0] = L.packed[1] = W->packed;
+    L.scales[0] = L.scales[1] = W->scales;
+    L.prefetch_ok = (W->flags & TERN_MATRIX_STATIC) ? 1 : 0;
+    L.q = q;
+    L.ldq = ldq;
+    L.s_x = s_x;
+    L.M = M;
+    L.residual = residual;
+    L.out = y;
+    L.ldo = ldy;
+    return run_gemv(L, "tern_gemv", static_cast<cudaStream_t>(stream));
+}
+
+tern_status tern_gateup_swiglu(const tern_matrix *Wg, const tern_matrix *Wu, const int8_t *q,
+                               int32_t ldq, const float *s_x, int32_t M, float *h, int32_t ldh,
+                               void *stream) {
+    tern_status st = check_matrix(Wg, "tern_gateup_swiglu (gate)");
+    if (st != TERN_OK) return st;
+    st = check_matrix(Wu, "tern_gateup_swiglu (up)");
+    if (st != TERN_OK) return st;
+    if (Wg->fmt != Wu->fmt || Wg->N != Wu->N || Wg->K != Wu->K || Wg->group != Wu->group ||
+        Wg->row_stride != Wu->row_stride)
+        return fail(TERN_EINVAL, "tern_gateup_swiglu: gate and up must share fmt, N, K, group, row_stride%s");
+    st = check_activations(q, ldq, Wg->K, s_x, M);
+    if (st != TERN_OK) return st;
+    if (!h || !aligned(h, 4) || ldh < Wg->N) return fail(TERN_EINVAL, "tern_gateup_swiglu: bad h or ldh%s");
+    tern::GemvLaunch L = {};
+    L.mode = tern::kModeSwiglu;
+    L.fmt = Wg->fmt;
+    L.N = Wg->N;
+    L.K = Wg->K;
+    L.G = static_cast<int>(tern::ceil_div(Wg->K, Wg->group));
+    L.row_bytes = tern::device_row_bytes(Wg->fmt, Wg->K);
+    L.row_stride = Wg->row_stride;
+    L.packed[0] = Wg->packed;
+    L.packed[1] = Wu->packed;
+    L.scales[0] = Wg->scales;
+    L.scales[1] = Wu->scales;
+    L.prefetch_ok = ((Wg->flags & Wu->flags) & TERN_MATRIX_STATIC) ? 1 : 0;
+    L.q = q;
+    L.ldq = ldq;
+    L.s_x = s_x;
+    L.M = M;
+    L.residual = nullptr;
+    L.out = h;
+    L.ldo = ldh;
+    return run_gemv(L, "tern_gateup_swiglu", static_cast<cudaStream_t>(stream));
+}
+
+tern_status tern_debug_group_partials(const tern_matrix *W, const int8_t *q, int32_t ldq, int32_t M,
+                                      int32_t *P, void *stream) {
+    tern_status st = check_matrix(W, "tern_debug_group_partials");
+    if (st != TERN_OK) return st;
+    if (M < 1 || M > 16) return fail(TERN_EINVAL, "tern_debug_group_partials: M must be in 1..16%s");
+    if (!q || !aligned(q, 16) || ldq < W->K || ldq % 16 != 0)
+        return fail(TERN_EINVAL, "tern_debug_group_partials: bad q or ldq%s");
+    if (!P || !aligned(P, 4)) return fail(TERN_EINVAL, "tern_debug_group_partials: bad P%s");
+    tern::GemvLaunch L = {};
+    L.mode = tern::kModePartials;
+    L.fmt = W->fmt;
+    L.N = W->N;
+    L.K = W->K;
+    L.G = static_cast<int>(tern::ceil_div(W->K, W->group));
+    L.row_bytes = tern::device_row_bytes(W->fmt, W->K);
+    L.row_stride = W->row_stride;
+    L.packed[0] = L.packed[1] = W->packed;
+    L.scales[0] = L.scales[1] = W->scales;
+    L.prefetch_ok = 0;
+    L.q = q;
+    L.ldq = ldq;
+    L.s_x = nullptr;
+    L.M = M;
+    L.out = P;
+    L.ldo = 0;
+    return run_gemv(L, "tern_debug_group_partials", static_cast<cudaStream_t>(stream));
+}
+
+tern_status tern_device_error(int32_t *code_out, void *stream) {
+    if (!code_out) return fail(TERN_EINVAL, "tern_device_error: null code_out%s");
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    int value = 0, zero = 0;
+    cudaError_t e = cudaMemcpyFromSymbolAsync(&value, tern::g_device_error, sizeof(int), 0,
+                                              cudaMemcpyDeviceToHost, s);
+    if (e == cudaSuccess)
+        e = cudaMemcpyToSymbolAsync(tern::g_device_error, &zero, sizeof(int), 0,
+                                    cudaMemcpyHostToDevice, s);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+    if (e != cudaSuccess) return cuda_status(e, "tern_device_error");
+    *code_out = value;
+    return TERN_OK;
+}
+
+}  // extern "C"

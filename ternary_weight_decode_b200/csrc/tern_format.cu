@@ -1,0 +1,255 @@
+// tern_format.cu -- load-time kernels: trits <-> device layout, canonical
+// file encodings <-> device layout (the load-time re-tile of the Bonsai page,
+// section "后面还有没有优化空间").  Not on the per-token hot path.
+//
+// Device layouts (see include/tern.h):
+//   D3: word w covers K in [20w, 20w+20); byte j holds K = 20w + j + 4i,
+//       i = 0..4, as y = ceil(256 V / 243), V = sum_i t_i 3^(4-i).
+//   D2: word w covers K in [16w, 16w+16); bits [2i,2i+1] of byte j hold t
+//       for K = 16w + 4i + j.
+// Canonical encodings:
+//   base-3: byte j = sum_{i<5} t_{5j+i} 3^i;  2-bit: byte j bits [2i,2i+1]
+//   = t_{4j+i}.  Both pad K with t = 1.
+#include "tern_internal.h"
+
+namespace tern {
+
+__device__ __forceinline__ int d3_encode(int V) { return (256 * V + 242) / 243; }
+
+// Returns V for a valid D3 code y, else -1.
+__device__ __forceinline__ int d3_decode(int y) {
+    int V = (243 * y) >> 8;
+    return (V <= 242 && d3_encode(V) == y) ? V : -1;
+}
+
+__device__ __forceinline__ int trit_digit(const int8_t *row, int64_t k, int K, int &bad) {
+    if (k >= K) return 1;
+    int t = row[k] + 1;
+    if (t < 0 || t > 2) {
+        ++bad;
+        return 1;
+    }
+    return t;
+}
+
+__global__ void pack_kernel(int fmt, const int8_t *__restrict__ trits, int N, int K,
+                            uint8_t *__restrict__ out, int64_t row_stride, int64_t used,
+                            int32_t *d_invalid) {
+    int64_t total = static_cast<int64_t>(N) * row_stride;
+    int bad = 0;
+    for (int64_t idx = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; idx < total;
+         idx += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+        int64_t n = idx / row_stride, b = idx % row_stride;
+        uint8_t code = 0;
+        if (b < used) {
+            const int8_t *row = trits + n * K;
+            int64_t wd = b >> 2;
+            int j = static_cast<int>(b & 3);
+            if (fmt == TERN_FMT_BASE3) {
+                int V = 0;
+                for (int i = 0; i < 5; ++i) V = 3 * V + trit_digit(row, 20 * wd + j + 4 * i, K, bad);
+                code = static_cast<uint8_t>(d3_encode(V));
+            } else {
+                int c = 0;
+                for (int i = 0; i < 4; ++i) c |= trit_digit(row, 16 * wd + 4 * i + j, K, bad) << (2 * i);
+                code = static_cast<uint8_t>(c);
+            }
+        }
+        out[idx] = code;
+    }
+    if (bad && d_invalid) atomicAdd(d_invalid, bad);
+}
+
+__global__ void unpack_kernel(int fmt, const uint8_t *__restrict__ packed, int N, int K,
+                              int64_t row_stride, int64_t used, int8_t *__restrict__ trits,
+                              int32_t *d_invalid) {
+    int64_t total = static_cast<int64_t>(N) * used;
+    int bad = 0;
+    for (int64_t idx = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; idx < total;
+         idx += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+        int64_t n = idx / used, b = idx % used;
+        int code = packed[n * row_stride + b];
+        int64_t wd = b >> 2;
+        int j = static_cast<int>(b & 3);
+        int8_t *row = trits + n * K;
+        if (fmt == TERN_FMT_BASE3) {
+            int V = d3_decode(code);
+            if (V < 0) {
+                ++bad;
+                V = 121;  // all digits 1 (w = 0)
+            }
+            for (int i = 4; i >= 0; --i) {  // digit 4 is the least significant
+                int t = V % 3;
+                V /= 3;
+                int64_t k = 20 * wd + j + 4 * i;
+                if (k < K)
+                    row[k] = static_cast<int8_t>(t - 1);
+                else if (t != 1)
+                    ++bad;
+            }
+        } else {
+            for (int i = 0; i < 4; ++i) {
+                int t = (code >> (2 * i)) & 3;
+                if (t == 3) {
+                    ++bad;
+                    t = 1;
+                }
+                int64_t k = 16 * wd + 4 * i + j;
+                if (k < K)
+                    row[k] = static_cast<int8_t>(t - 1);
+                else if (t != 1)
+                    ++bad;
+            }
+        }
+    }
+    if (bad && d_invalid) atomicAdd(d_invalid, bad);
+}
+
+// Digit t (0..2) of canonical position k of a row; counts invalid codes and
+// (for positions past K) padding digits other than 1.
+__device__ __forceinline__ int canonical_digit(int fmt, const uint8_t *row, int64_t k, int K,
+                                               int64_t cbytes, int &bad) {
+    int per = (fmt == TERN_FMT_BASE3) ? 5 : 4;
+    int64_t byte = k / per;
+    if (byte >= cbytes) return 1;  // beyond the canonical row: padding of the device layout
+    int code = row[byte];
+    int i = static_cast<int>(k % per);
+    int t;
+    if (fmt == TERN_FMT_BASE3) {
+        if (code >= 243) {
+            ++bad;
+            return 1;
+        }
+        for (int s = 0; s < i; ++s) code /= 3;
+        t = code % 3;
+    } else {
+        t = (code >> (2 * i)) & 3;
+        if (t == 3) {
+            ++bad;
+            return 1;
+        }
+    }
+    if (k >= K) {
+        if (t != 1) ++bad;
+        return 1;
+    }
+    return t;
+}
+
+__global__ void import_kernel(int fmt, const uint8_t *__restrict__ canon, int N, int K,
+                              int64_t cbytes, uint8_t *__restrict__ out, int64_t row_stride,
+                              int64_t used, int32_t *d_invalid) {
+    int64_t total = static_cast<int64_t>(N) * row_stride;
+    int bad = 0;
+    for (int64_t idx = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; idx < total;
+         idx += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+        int64_t n = idx / row_stride, b = idx % row_stride;
+        uint8_t code = 0;
+        if (b < used) {
+            const uint8_t *row = canon + n * cbytes;
+            int64_t wd = b >> 2;
+            int j = static_cast<int>(b & 3);
+            if (fmt == TERN_FMT_BASE3) {
+                int V = 0;
+                for (int i = 0; i < 5; ++i)
+                    V = 3 * V + canonical_digit(fmt, row, 20 * wd + j + 4 * i, K, cbytes, bad);
+                code = static_cast<uint8_t>(d3_encode(V));
+            } else {
+                int c = 0;
+                for (int i = 0; i < 4; ++i)
+                    c |= canonical_digit(fmt, row, 16 * wd + 4 * i + j, K, cbytes, bad) << (2 * i);
+                code = static_cast<uint8_t>(c);
+            }
+        }
+        out[idx] = code;
+    }
+    if (bad && d_invalid) atomicAdd(d_invalid, bad);
+}
+
+// Digit t of position k < K of a device-layout row.
+__device__ __forceinline__ int device_digit(int fmt, const uint8_t *row, int64_t k, int &bad) {
+    if (fmt == TERN_FMT_BASE3) {
+        int64_t wd = k / 20;
+        int r = static_cast<int>(k % 20);
+        int j = r & 3, i = r >> 2;
+        int V = d3_decode(row[4 * wd + j]);
+        if (V < 0) {
+            ++bad;
+            return 1;
+        }
+        for (int s = i; s < 4; ++s) V /= 3;  // digit i has weight 3^(4-i)
+        return V % 3;
+    }
+    int64_t wd = k / 16;
+    int r = static_cast<int>(k % 16);
+    int j = r & 3, i = r >> 2;
+    int t = (row[4 * wd + j] >> (2 * i)) & 3;
+    if (t == 3) {
+        ++bad;
+        return 1;
+    }
+    return t;
+}
+
+__global__ void export_kernel(int fmt, const uint8_t *__restrict__ packed, int N, int K,
+                              int64_t row_stride, uint8_t *__restrict__ canon, int64_t cbytes,
+                              int32_t *d_invalid) {
+    int64_t total = static_cast<int64_t>(N) * cbytes;
+    int per = (fmt == TERN_FMT_BASE3) ? 5 : 4;
+    int bad = 0;
+    for (int64_t idx = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; idx < total;
+         idx += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+        int64_t n = idx / cbytes, cb = idx % cbytes;
+        const uint8_t *row = packed + n * row_stride;
+        int value = 0;
+        for (int i = per - 1; i >= 0; --i) {
+            int64_t k = cb * per + i;
+            int t = (k < K) ? device_digit(fmt, row, k, bad) : 1;
+            value = (fmt == TERN_FMT_BASE3) ? value * 3 + t : (value << 2) | t;
+        }
+        canon[idx] = static_cast<uint8_t>(value);
+    }
+    if (bad && d_invalid) atomicAdd(d_invalid, bad);
+}
+
+static int grid_for(int64_t total) {
+    int64_t blocks = (total + 255) / 256;
+    if (blocks < 1) blocks = 1;
+    if (blocks > 148 * 64) blocks = 148 * 64;
+    return static_cast<int>(blocks);
+}
+
+cudaError_t launch_pack(int fmt, const int8_t *trits, int N, int K, void *out, int64_t row_stride,
+                        int32_t *d_invalid, cudaStream_t s) {
+    int64_t used = device_row_bytes(fmt, K);
+    pack_kernel<<<grid_for(static_cast<int64_t>(N) * row_stride), 256, 0, s>>>(
+        fmt, trits, N, K, static_cast<uint8_t *>(out), row_stride, used, d_invalid);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_unpack(int fmt, const void *packed, int N, int K, int64_t row_stride,
+                          int8_t *trits, int32_t *d_invalid, cudaStream_t s) {
+    int64_t used = device_row_bytes(fmt, K);
+    unpack_kernel<<<grid_for(static_cast<int64_t>(N) * used), 256, 0, s>>>(
+        fmt, static_cast<const uint8_t *>(packed), N, K, row_stride, used, trits, d_invalid);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_import(int fmt, const uint8_t *canon, int N, int K, void *out,
+                          int64_t row_stride, int32_t *d_invalid, cudaStream_t s) {
+    int64_t used = device_row_bytes(fmt, K);
+    int64_t cbytes = canonical_row_bytes(fmt, K);
+    import_kernel<<<grid_for(static_cast<int64_t>(N) * row_stride), 256, 0, s>>>(
+        fmt, canon, N, K, cbytes, static_cast<uint8_t *>(out), row_stride, used, d_invalid);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_export(int fmt, const void *packed, int N, int K, int64_t row_stride,
+                          uint8_t *canon, int32_t *d_invalid, cudaStream_t s) {
+    int64_t cbytes = canonical_row_bytes(fmt, K);
+    export_kernel<<<grid_for(static_cast<int64_t>(N) * cbytes), 256, 0, s>>>(
+        fmt, static_cast<const uint8_t *>(packed), N, K, row_stride, canon, cbytes, d_invalid);
+    return cudaGetLastError();
+}
+
+}  // namespace tern

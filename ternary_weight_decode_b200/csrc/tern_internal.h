@@ -1,0 +1,64 @@
+// tern_internal.h -- declarations shared between the C-ABI layer and the
+// kernel launchers of libtern (not installed; the public ABI is tern.h).
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/tern.h"
+
+namespace tern {
+
+inline int64_t device_row_bytes(int fmt, int64_t K) {
+    if (fmt == TERN_FMT_BASE3) return 4 * ((K + 19) / 20);
+    if (fmt == TERN_FMT_2BIT) return 4 * ((K + 15) / 16);
+    return -1;
+}
+
+inline int64_t canonical_row_bytes(int fmt, int64_t K) {
+    if (fmt == TERN_FMT_BASE3) return (K + 4) / 5;
+    if (fmt == TERN_FMT_2BIT) return (K + 3) / 4;
+    return -1;
+}
+
+inline int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
+
+// ---------------------------------------------------------------- format
+cudaError_t launch_pack(int fmt, const int8_t *trits, int N, int K, void *out, int64_t row_stride,
+                        int32_t *d_invalid, cudaStream_t s);
+cudaError_t launch_unpack(int fmt, const void *packed, int N, int K, int64_t row_stride,
+                          int8_t *trits, int32_t *d_invalid, cudaStream_t s);
+cudaError_t launch_import(int fmt, const uint8_t *canon, int N, int K, void *out,
+                          int64_t row_stride, int32_t *d_invalid, cudaStream_t s);
+cudaError_t launch_export(int fmt, const void *packed, int N, int K, int64_t row_stride,
+                          uint8_t *canon, int32_t *d_invalid, cudaStream_t s);
+
+// ---------------------------------------------------------------- quant
+cudaError_t launch_act_quant(const void *x, bool fp16, int M, int K, int ldx, int fwht_block,
+                             int flags, int8_t *q, int ldq, float *s_x, cudaStream_t s);
+
+// ---------------------------------------------------------------- gemv
+enum GemvMode : int { kModeGemv = 0, kModeSwiglu = 1, kModePartials = 2 };
+
+struct GemvLaunch {
+    int mode;
+    int fmt;
+    int N, K, G;
+    int64_t row_bytes;  // used bytes per row (the TMA box's x extent)
+    int64_t row_stride;
+    const void *packed[2];
+    const uint16_t *scales[2];
+    int prefetch_ok;  // both matrices carry TERN_MATRIX_STATIC
+    const int8_t *q;
+    int ldq;
+    const float *s_x;
+    int M;
+    const float *residual;
+    void *out;  // y, h (fp32) or partials (int32)
+    int ldo;
+};
+
+cudaError_t launch_gemv(const GemvLaunch &L, cudaStream_t s, const char **why);
+
+}  // namespace tern

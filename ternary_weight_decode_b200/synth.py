@@ -20,7 +20,7 @@ of the single-GEMV workload).  A group scale is drawn from ``u24 = h >> 40``
 as ``fp16(fp32(fp32(u24 * 2**-24) * 0.045) + 0.005)`` with every fp32 step
 rounded to nearest, giving scales in [0.005, 0.05).
 
-The device generator in ``csrc/synth.cu`` implements the same definition;
+The device generator in ``synth_csrc/tern_synth.cu`` implements the same definition;
 a GPU test checks the two bit for bit.
 
 Activations are drawn on the host with numpy's PCG64: N(0, 1), 1% of the
@@ -35,8 +35,8 @@ MASK64 = (1 << 64) - 1
 T_NEG = 1288490189  # ceil(0.3 * 2**32)
 T_POS = 3006477108  # ceil(0.7 * 2**32)
 
-# Stream ids: projection p of layer l uses streams STREAM_BASE(l, p) (trits)
-# and STREAM_BASE(l, p) + 1 (scales).
+# Stream ids: projection p of layer l draws its trits from stream_id(l, p)
+# and its scales from stream_id(l, p, scales=True).
 PROJ_QKV, PROJ_O, PROJ_GATE, PROJ_UP, PROJ_DOWN = 0, 1, 2, 3, 4
 
 
@@ -122,3 +122,56 @@ def activation_rows(seeds, K: int) -> np.ndarray:
 
 def groups(K: int, group: int = 128) -> int:
     return (K + group - 1) // group
+
+
+# ---------------------------------------------------------------- device side
+_synth_lib = None
+
+
+def _device_lib():
+    """libtern_synth.so: the same generator as above, run on the GPU."""
+    global _synth_lib
+    if _synth_lib is None:
+        import ctypes
+        import os
+        path = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libtern_synth.so")
+        if not os.path.exists(path):
+            raise RuntimeError(f"{path} is missing: build it with "
+                               "`python -m ternary_weight_decode_b200.build`")
+        L = ctypes.CDLL(path)
+        L.tern_synth_trits.restype = ctypes.c_int
+        L.tern_synth_trits.argtypes = [ctypes.c_uint64, ctypes.c_int64, ctypes.c_int64,
+                                       ctypes.c_int64, ctypes.c_void_p, ctypes.c_void_p]
+        L.tern_synth_scales.restype = ctypes.c_int
+        L.tern_synth_scales.argtypes = [ctypes.c_uint64, ctypes.c_int64, ctypes.c_int64,
+                                        ctypes.c_void_p, ctypes.c_void_p]
+        _synth_lib = L
+    return _synth_lib
+
+
+def device_trits(seed: int, stream: int, N: int, K: int, out=None, row0: int = 0):
+    """Trits of rows [row0, row0+N) as a CUDA int8 tensor [N, K]."""
+    import ctypes
+    import torch
+    if out is None:
+        out = torch.empty((N, K), dtype=torch.int8, device="cuda")
+    rc = _device_lib().tern_synth_trits(stream_key(seed, stream), row0, N, K,
+                                        ctypes.c_void_p(out.data_ptr()),
+                                        ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
+    if rc != 0:
+        raise RuntimeError(f"tern_synth_trits failed with CUDA error {rc}")
+    return out
+
+
+def device_scales(seed: int, stream: int, N: int, G: int, out=None):
+    """fp16 group scales as a CUDA float16 tensor [N, G]."""
+    import ctypes
+    import torch
+    if out is None:
+        out = torch.empty((N, G), dtype=torch.float16, device="cuda")
+    rc = _device_lib().tern_synth_scales(stream_key(seed, stream), N, G,
+                                         ctypes.c_void_p(out.data_ptr()),
+                                         ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
+    if rc != 0:
+        raise RuntimeError(f"tern_synth_scales failed with CUDA error {rc}")
+    return out

@@ -1,0 +1,233 @@
+"""Python binding of libtern.so (include/tern.h): argument marshalling only.
+
+Every function has the name of its C entry point, takes torch CUDA tensors
+for device buffers, passes their pointers and the current torch stream, and
+raises ``TernError`` on a non-OK status.  All arithmetic runs in the CUDA
+kernels of libtern.so; there is no CPU fallback and no other backend: when
+the library is missing this module raises instead of computing anything.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+from dataclasses import dataclass
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libtern.so")
+
+TERN_OK, TERN_EINVAL, TERN_ECUDA, TERN_EUNSUPPORTED, TERN_ETIMEOUT = 0, 1, 2, 3, 4
+TERN_FMT_BASE3, TERN_FMT_2BIT = 0, 1
+TERN_MATRIX_STATIC = 1
+TERN_QUANT_RMSNORM = 1
+GROUP = 128
+
+
+class TernError(RuntimeError):
+    def __init__(self, status: int, where: str, message: str):
+        super().__init__(f"{where}: status {status}: {message}")
+        self.status = status
+
+
+class tern_matrix(ctypes.Structure):
+    _fields_ = [
+        ("fmt", ctypes.c_int32),
+        ("N", ctypes.c_int32),
+        ("K", ctypes.c_int32),
+        ("group", ctypes.c_int32),
+        ("row_stride", ctypes.c_int64),
+        ("packed", ctypes.c_void_p),
+        ("scales", ctypes.c_void_p),
+        ("flags", ctypes.c_int32),
+        ("reserved", ctypes.c_int32),
+    ]
+
+
+_lib = None
+_lock = threading.Lock()
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded libtern.so; raises when it has not been built."""
+    global _lib
+    with _lock:
+        if _lib is None:
+            if not os.path.exists(LIB_PATH):
+                raise RuntimeError(
+                    f"{LIB_PATH} is missing: build it with "
+                    "`python -m ternary_weight_decode_b200.build` (no CPU fallback exists)")
+            L = ctypes.CDLL(LIB_PATH)
+            i32, i64, p, sz = ctypes.c_int32, ctypes.c_int64, ctypes.c_void_p, ctypes.c_size_t
+            pm = ctypes.POINTER(tern_matrix)
+            sig = {
+                "tern_status_string": (ctypes.c_char_p, [ctypes.c_int]),
+                "tern_last_error": (ctypes.c_char_p, []),
+                "tern_packed_size": (ctypes.c_int, [i32, i32, i32, i32, ctypes.POINTER(i64),
+                                                    ctypes.POINTER(sz), ctypes.POINTER(sz)]),
+                "tern_canonical_row_bytes": (ctypes.c_int, [i32, i32, ctypes.POINTER(i64)]),
+                "tern_pack": (ctypes.c_int, [i32, p, i32, i32, p, i64, p, p]),
+                "tern_unpack": (ctypes.c_int, [pm, p, p, p]),
+                "tern_import": (ctypes.c_int, [i32, p, i32, i32, p, i64, p, p]),
+                "tern_export": (ctypes.c_int, [pm, p, p, p]),
+                "act_quant_fwht": (ctypes.c_int, [p, i32, i32, i32, i32, i32, i32, p, i32, p, p]),
+                "tern_gemv": (ctypes.c_int, [pm, p, i32, p, i32, p, p, i32, p]),
+                "tern_gateup_swiglu": (ctypes.c_int, [pm, pm, p, i32, p, i32, p, i32, p]),
+                "tern_debug_group_partials": (ctypes.c_int, [pm, p, i32, i32, p, p]),
+                "tern_device_error": (ctypes.c_int, [ctypes.POINTER(i32), p]),
+            }
+            for name, (res, args) in sig.items():
+                f = getattr(L, name)
+                f.restype = res
+                f.argtypes = args
+            _lib = L
+    return _lib
+
+
+def _check(status: int, where: str) -> None:
+    if status != TERN_OK:
+        msg = lib().tern_last_error().decode(errors="replace")
+        raise TernError(status, where, msg)
+
+
+def _ptr(t):
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError("device buffers must be CUDA tensors")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream=None):
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+# ------------------------------------------------------------------ sizes
+def tern_packed_size(fmt: int, N: int, K: int, group: int = GROUP):
+    rs = ctypes.c_int64()
+    pb = ctypes.c_size_t()
+    sb = ctypes.c_size_t()
+    _check(lib().tern_packed_size(fmt, N, K, group, ctypes.byref(rs), ctypes.byref(pb),
+                                  ctypes.byref(sb)), "tern_packed_size")
+    return rs.value, pb.value, sb.value
+
+
+def tern_canonical_row_bytes(fmt: int, K: int) -> int:
+    b = ctypes.c_int64()
+    _check(lib().tern_canonical_row_bytes(fmt, K, ctypes.byref(b)), "tern_canonical_row_bytes")
+    return b.value
+
+
+# ------------------------------------------------------------------ matrices
+@dataclass
+class TernMatrix:
+    """A packed device matrix: `packed` uint8 [N, row_stride], `scales` fp16 [N, G]."""
+    fmt: int
+    N: int
+    K: int
+    row_stride: int
+    packed: torch.Tensor
+    scales: torch.Tensor
+    static: bool = True
+
+    def struct(self) -> tern_matrix:
+        return tern_matrix(self.fmt, self.N, self.K, GROUP, self.row_stride,
+                           self.packed.data_ptr(), self.scales.data_ptr(),
+                           TERN_MATRIX_STATIC if self.static else 0, 0)
+
+    @staticmethod
+    def empty(fmt: int, N: int, K: int, device="cuda") -> "TernMatrix":
+        rs, pb, sb = tern_packed_size(fmt, N, K)
+        packed = torch.empty((N, rs), dtype=torch.uint8, device=device)
+        scales = torch.empty((N, (K + GROUP - 1) // GROUP), dtype=torch.float16, device=device)
+        return TernMatrix(fmt, N, K, rs, packed, scales)
+
+
+def tern_pack(fmt: int, trits: torch.Tensor, out: TernMatrix, d_invalid=None, stream=None):
+    N, K = trits.shape
+    assert trits.dtype == torch.int8 and trits.is_contiguous()
+    assert out.packed.dtype == torch.uint8 and out.packed.shape == (N, out.row_stride)
+    _check(lib().tern_pack(fmt, _ptr(trits), N, K, _ptr(out.packed), out.row_stride,
+                           _ptr(d_invalid), _stream(stream)), "tern_pack")
+
+
+def tern_unpack(W: TernMatrix, trits_out: torch.Tensor, d_invalid=None, stream=None):
+    assert trits_out.dtype == torch.int8 and trits_out.shape == (W.N, W.K)
+    s = W.struct()
+    _check(lib().tern_unpack(ctypes.byref(s), _ptr(trits_out), _ptr(d_invalid), _stream(stream)),
+           "tern_unpack")
+
+
+def tern_import(fmt: int, canonical: torch.Tensor, K: int, out: TernMatrix, d_invalid=None,
+                stream=None):
+    N = canonical.shape[0]
+    assert canonical.dtype == torch.uint8 and canonical.is_contiguous()
+    assert canonical.shape[1] == tern_canonical_row_bytes(fmt, K)
+    _check(lib().tern_import(fmt, _ptr(canonical), N, K, _ptr(out.packed), out.row_stride,
+                             _ptr(d_invalid), _stream(stream)), "tern_import")
+
+
+def tern_export(W: TernMatrix, canonical_out: torch.Tensor, d_invalid=None, stream=None):
+    assert canonical_out.dtype == torch.uint8
+    assert canonical_out.shape == (W.N, tern_canonical_row_bytes(W.fmt, W.K))
+    s = W.struct()
+    _check(lib().tern_export(ctypes.byref(s), _ptr(canonical_out), _ptr(d_invalid),
+                             _stream(stream)), "tern_export")
+
+
+# ------------------------------------------------------------------ compute
+def act_quant_fwht(x: torch.Tensor, q: torch.Tensor, s_x: torch.Tensor, fwht_block: int = 0,
+                   K: int | None = None, flags: int = 0, stream=None):
+    """x fp16/fp32 [M, ldx] -> q int8 [M, ldq], s_x fp32 [M] (first K columns of x)."""
+    assert x.dtype in (torch.float16, torch.float32) and x.stride(1) == 1
+    M = x.shape[0]
+    K = x.shape[1] if K is None else K
+    assert q.dtype == torch.int8 and q.stride(1) == 1 and q.shape[0] == M
+    assert s_x.dtype == torch.float32 and s_x.numel() >= M
+    _check(lib().act_quant_fwht(_ptr(x), 1 if x.dtype == torch.float16 else 0, M, K, x.stride(0),
+                                fwht_block, flags, _ptr(q), q.stride(0), _ptr(s_x),
+                                _stream(stream)),
+           "act_quant_fwht")
+
+
+def tern_gemv(W: TernMatrix, q: torch.Tensor, s_x: torch.Tensor, y: torch.Tensor,
+              residual: torch.Tensor | None = None, M: int | None = None, stream=None):
+    M = q.shape[0] if M is None else M
+    assert q.dtype == torch.int8 and y.dtype == torch.float32 and y.stride(1) == 1
+    if residual is not None:
+        assert residual.dtype == torch.float32 and residual.stride(0) == y.stride(0)
+    s = W.struct()
+    _check(lib().tern_gemv(ctypes.byref(s), _ptr(q), q.stride(0), _ptr(s_x), M, _ptr(residual),
+                           _ptr(y), y.stride(0), _stream(stream)), "tern_gemv")
+
+
+def tern_gateup_swiglu(Wg: TernMatrix, Wu: TernMatrix, q: torch.Tensor, s_x: torch.Tensor,
+                       h: torch.Tensor, M: int | None = None, stream=None):
+    M = q.shape[0] if M is None else M
+    assert q.dtype == torch.int8 and h.dtype == torch.float32 and h.stride(1) == 1
+    sg, su = Wg.struct(), Wu.struct()
+    _check(lib().tern_gateup_swiglu(ctypes.byref(sg), ctypes.byref(su), _ptr(q), q.stride(0),
+                                    _ptr(s_x), M, _ptr(h), h.stride(0), _stream(stream)),
+           "tern_gateup_swiglu")
+
+
+def tern_debug_group_partials(W: TernMatrix, q: torch.Tensor, P: torch.Tensor,
+                              M: int | None = None, stream=None):
+    M = q.shape[0] if M is None else M
+    assert P.dtype == torch.int32 and P.is_contiguous()
+    s = W.struct()
+    _check(lib().tern_debug_group_partials(ctypes.byref(s), _ptr(q), q.stride(0), M, _ptr(P),
+                                           _stream(stream)), "tern_debug_group_partials")
+
+
+def tern_device_error(stream=None) -> int:
+    code = ctypes.c_int32()
+    _check(lib().tern_device_error(ctypes.byref(code), _stream(stream)), "tern_device_error")
+    return code.value
+
+
+def loaded_library_path() -> str:
+    lib()
+    return LIB_PATH

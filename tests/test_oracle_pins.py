@@ -200,6 +200,18 @@ def test_quant_fwht_dequantises_to_orthonormal_hadamard():
     assert (err <= s[:, None] * 0.5 * (1 + 1e-4) + 1e-6).all()
 
 
+def test_quant_rmsnorm_scales_by_inverse_rms():
+    x = synth.activations(13, 3, 640).astype(np.float32)
+    q, s = oracle.act_quant(x)
+    qn, sn = oracle.act_quant(x, rmsnorm=True)
+    np.testing.assert_array_equal(q, qn)
+    rms = np.sqrt((x.astype(np.float64) ** 2).mean(axis=1) + 1e-6)
+    np.testing.assert_allclose(sn, s / rms, rtol=1e-7)
+    # a constant row of value c has rms |c|: the scale becomes 1/127
+    qc, sc = oracle.act_quant(np.full((1, 256), -3.0, np.float32), rmsnorm=True)
+    np.testing.assert_allclose(sc[0], 1 / 127, rtol=1e-6)
+
+
 def test_quant_rejects_bad_arguments():
     with pytest.raises(oracle.OracleError):
         oracle.act_quant(np.ones((1, 200), np.float32), fwht_block=128)
