@@ -62,6 +62,11 @@ typedef enum {
  * the scale, s_x *= fp32(1/sqrt(mean_k x_k^2 + 1e-6)); q is unchanged. */
 #define TERN_QUANT_RMSNORM 1
 
+/* Fused-quantisation flag (tern_gemv_fused, tern_gateup_swiglu_fused): rotate
+ * the input by the 128-point Hadamard transform before quantising it, exactly
+ * as act_quant_fwht with fwht_block = 128. */
+#define TERN_QUANT_FWHT128 2
+
 /*
  * A packed weight matrix W [N][K] in the device layout written by tern_pack
  * or tern_import:
@@ -191,6 +196,47 @@ tern_status tern_gateup_swiglu(const tern_matrix *Wg, const tern_matrix *Wu,
 tern_status tern_debug_group_partials(const tern_matrix *W, const int8_t *q,
                                       int32_t ldq, int32_t M, int32_t *P,
                                       void *stream);
+
+/*
+ * Activation statistics, the input of the fused quantisation below.  For each
+ * token row m of x (fp32 [M][ldx], 16-byte aligned, ldx % 4 == 0) and each
+ * 128-element block b of its first K elements (the last block zero-padded):
+ *   stats[(m*stats_ld + b)*4 + 0] = max |x_b|
+ *   stats[(m*stats_ld + b)*4 + 1] = max |H x_b|   (H: act_quant_fwht's rotation)
+ *   stats[(m*stats_ld + b)*4 + 2] = sum x_b^2     (fp32)
+ *   stats[(m*stats_ld + b)*4 + 3] = 0
+ * stats: device fp32, 16-byte aligned, stats_ld >= ceil(K/128).
+ */
+tern_status tern_act_stats(const float *x, int32_t M, int32_t K, int32_t ldx,
+                           float *stats, int32_t stats_ld, void *stream);
+
+/*
+ * tern_gemv with the per-token quantisation of its input done inside the
+ * kernel: x is the fp32 activation [M][ldx] (16-byte aligned, ldx % 4 == 0,
+ * ldx >= K; must not overlap y), x_stats its block statistics (as written by
+ * tern_act_stats, or by the y_stats of the call that produced x; row stride
+ * x_stats_ld blocks).  With qflags TERN_QUANT_FWHT128 and/or
+ * TERN_QUANT_RMSNORM, q and s_x are those act_quant_fwht(x, fwht_block =
+ * 128 if FWHT128, flags = RMSNORM) gives -- q bit for bit; s_x with RMSNORM
+ * up to the summation order of the squares.  Then y as tern_gemv computes
+ * it.  y_stats (optional, 16-byte aligned, y_stats_ld >= ceil(N/128)) receives
+ * the statistics of y, so the next call can quantise y without a separate
+ * launch (the Bonsai page's chain of re-quantised activations).
+ */
+tern_status tern_gemv_fused(const tern_matrix *W, const float *x, int32_t ldx,
+                            const float *x_stats, int32_t x_stats_ld,
+                            int32_t qflags, int32_t M, const float *residual,
+                            float *y, int32_t ldy, float *y_stats,
+                            int32_t y_stats_ld, void *stream);
+
+/* tern_gateup_swiglu with the fused input quantisation of tern_gemv_fused;
+ * h_stats (optional) receives the statistics of h. */
+tern_status tern_gateup_swiglu_fused(const tern_matrix *Wg, const tern_matrix *Wu,
+                                     const float *x, int32_t ldx,
+                                     const float *x_stats, int32_t x_stats_ld,
+                                     int32_t qflags, int32_t M, float *h,
+                                     int32_t ldh, float *h_stats,
+                                     int32_t h_stats_ld, void *stream);
 
 /*
  * Reads and clears the device error word of the current device: 0 when no

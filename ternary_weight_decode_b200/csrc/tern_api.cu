@@ -257,17 +257,116 @@ tern_status tern_debug_group_partials(const tern_matrix *W, const int8_t *q, int
 
 tern_status tern_device_error(int32_t *code_out, void *stream) {
     if (!code_out) return fail(TERN_EINVAL, "tern_device_error: null code_out%s");
-    cudaStream_t s = static_cast<cudaStream_t>(stream);
-    int value = 0, zero = 0;
-    cudaError_t e = cudaMemcpyFromSymbolAsync(&value, tern::g_device_error, sizeof(int), 0,
-                                              cudaMemcpyDeviceToHost, s);
-    if (e == cudaSuccess)
-        e = cudaMemcpyToSymbolAsync(tern::g_device_error, &zero, sizeof(int), 0,
-                                    cudaMemcpyHostToDevice, s);
-    if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+    int value = 0;
+    cudaError_t e = tern::read_clear_device_error(&value, static_cast<cudaStream_t>(stream));
     if (e != cudaSuccess) return cuda_status(e, "tern_device_error");
     *code_out = value;
     return TERN_OK;
+}
+
+tern_status tern_act_stats(const float *x, int32_t M, int32_t K, int32_t ldx, float *stats,
+                           int32_t stats_ld, void *stream) {
+    if (M < 1 || K < 1) return fail(TERN_EINVAL, "tern_act_stats: M and K must be >= 1%s");
+    if (!x || !aligned(x, 16) || ldx < K || ldx % 4 != 0)
+        return fail(TERN_EINVAL, "tern_act_stats: x must be 16-byte aligned, ldx >= K, ldx %% 4 == 0%s");
+    if (!stats || !aligned(stats, 16) || stats_ld < tern::ceil_div(K, 128))
+        return fail(TERN_EINVAL, "tern_act_stats: bad stats or stats_ld%s");
+    return cuda_status(tern::launch_act_stats(x, M, K, ldx, stats, stats_ld,
+                                              static_cast<cudaStream_t>(stream)),
+                       "tern_act_stats");
+}
+
+static tern_status check_fused_input(const float *x, int32_t ldx, int32_t K, const float *x_stats,
+                                     int32_t x_stats_ld, int32_t qflags, int32_t M) {
+    if (M < 1 || M > 16) return fail(TERN_EINVAL, "fused: M must be in 1..16%s");
+    if (!x || !aligned(x, 16) || ldx < K || ldx % 4 != 0)
+        return fail(TERN_EINVAL, "fused: x must be 16-byte aligned, ldx >= K, ldx %% 4 == 0%s");
+    if (!x_stats || !aligned(x_stats, 16) || x_stats_ld < tern::ceil_div(K, 128))
+        return fail(TERN_EINVAL, "fused: bad x_stats or x_stats_ld%s");
+    if (qflags & ~(TERN_QUANT_FWHT128 | TERN_QUANT_RMSNORM))
+        return fail(TERN_EINVAL, "fused: unknown qflags bits%s");
+    if ((qflags & TERN_QUANT_FWHT128) && K % 128 != 0)
+        return fail(TERN_EINVAL, "fused: the Hadamard rotation needs K %% 128 == 0%s");
+    return TERN_OK;
+}
+
+tern_status tern_gemv_fused(const tern_matrix *W, const float *x, int32_t ldx, const float *x_stats,
+                            int32_t x_stats_ld, int32_t qflags, int32_t M, const float *residual,
+                            float *y, int32_t ldy, float *y_stats, int32_t y_stats_ld,
+                            void *stream) {
+    tern_status st = check_matrix(W, "tern_gemv_fused");
+    if (st != TERN_OK) return st;
+    st = check_fused_input(x, ldx, W->K, x_stats, x_stats_ld, qflags, M);
+    if (st != TERN_OK) return st;
+    if (!y || !aligned(y, 4) || ldy < W->N) return fail(TERN_EINVAL, "tern_gemv_fused: bad y or ldy%s");
+    if (residual && !aligned(residual, 4)) return fail(TERN_EINVAL, "tern_gemv_fused: bad residual%s");
+    if (y_stats && (!aligned(y_stats, 16) || y_stats_ld < tern::ceil_div(W->N, 128)))
+        return fail(TERN_EINVAL, "tern_gemv_fused: bad y_stats or y_stats_ld%s");
+    tern::GemvLaunch L = {};
+    L.mode = tern::kModeGemv;
+    L.fmt = W->fmt;
+    L.N = W->N;
+    L.K = W->K;
+    L.G = static_cast<int>(tern::ceil_div(W->K, W->group));
+    L.row_bytes = tern::device_row_bytes(W->fmt, W->K);
+    L.row_stride = W->row_stride;
+    L.packed[0] = L.packed[1] = W->packed;
+    L.scales[0] = L.scales[1] = W->scales;
+    L.prefetch_ok = (W->flags & TERN_MATRIX_STATIC) ? 1 : 0;
+    L.M = M;
+    L.residual = residual;
+    L.out = y;
+    L.ldo = ldy;
+    L.x = x;
+    L.ldx = ldx;
+    L.x_stats = x_stats;
+    L.x_stats_ld = x_stats_ld;
+    L.qflags = qflags;
+    L.y_stats = y_stats;
+    L.y_stats_ld = y_stats_ld;
+    return run_gemv(L, "tern_gemv_fused", static_cast<cudaStream_t>(stream));
+}
+
+tern_status tern_gateup_swiglu_fused(const tern_matrix *Wg, const tern_matrix *Wu, const float *x,
+                                     int32_t ldx, const float *x_stats, int32_t x_stats_ld,
+                                     int32_t qflags, int32_t M, float *h, int32_t ldh,
+                                     float *h_stats, int32_t h_stats_ld, void *stream) {
+    tern_status st = check_matrix(Wg, "tern_gateup_swiglu_fused (gate)");
+    if (st != TERN_OK) return st;
+    st = check_matrix(Wu, "tern_gateup_swiglu_fused (up)");
+    if (st != TERN_OK) return st;
+    if (Wg->fmt != Wu->fmt || Wg->N != Wu->N || Wg->K != Wu->K || Wg->group != Wu->group ||
+        Wg->row_stride != Wu->row_stride)
+        return fail(TERN_EINVAL, "tern_gateup_swiglu_fused: gate and up must share fmt, N, K, group, row_stride%s");
+    st = check_fused_input(x, ldx, Wg->K, x_stats, x_stats_ld, qflags, M);
+    if (st != TERN_OK) return st;
+    if (!h || !aligned(h, 4) || ldh < Wg->N) return fail(TERN_EINVAL, "tern_gateup_swiglu_fused: bad h or ldh%s");
+    if (h_stats && (!aligned(h_stats, 16) || h_stats_ld < tern::ceil_div(Wg->N, 128)))
+        return fail(TERN_EINVAL, "tern_gateup_swiglu_fused: bad h_stats or h_stats_ld%s");
+    tern::GemvLaunch L = {};
+    L.mode = tern::kModeSwiglu;
+    L.fmt = Wg->fmt;
+    L.N = Wg->N;
+    L.K = Wg->K;
+    L.G = static_cast<int>(tern::ceil_div(Wg->K, Wg->group));
+    L.row_bytes = tern::device_row_bytes(Wg->fmt, Wg->K);
+    L.row_stride = Wg->row_stride;
+    L.packed[0] = Wg->packed;
+    L.packed[1] = Wu->packed;
+    L.scales[0] = Wg->scales;
+    L.scales[1] = Wu->scales;
+    L.prefetch_ok = ((Wg->flags & Wu->flags) & TERN_MATRIX_STATIC) ? 1 : 0;
+    L.M = M;
+    L.out = h;
+    L.ldo = ldh;
+    L.x = x;
+    L.ldx = ldx;
+    L.x_stats = x_stats;
+    L.x_stats_ld = x_stats_ld;
+    L.qflags = qflags;
+    L.y_stats = h_stats;
+    L.y_stats_ld = h_stats_ld;
+    return run_gemv(L, "tern_gateup_swiglu_fused", static_cast<cudaStream_t>(stream));
 }
 
 }  // extern "C"

@@ -145,4 +145,62 @@ __device__ __forceinline__ uint4 lds128(const void *p) {
     return *reinterpret_cast<const uint4 *>(p);
 }
 
+// ---------------------------------------------------------------- Hadamard
+// Unnormalised 128-point Sylvester Hadamard transform of one block held by a
+// warp, lane l owning elements 4l..4l+3 in r[0..3]: radix-2 butterflies
+// (a, b) -> (a + b, a - b) in stage order h = 1, 2, 4, ..., 64, each output a
+// single fp32 add or subtract.  Every kernel that rotates uses this routine,
+// so all of them produce the same bits.
+__device__ __forceinline__ void fwht128_warp(float (&r)[4], int lane) {
+    float a0 = __fadd_rn(r[0], r[1]), a1 = __fsub_rn(r[0], r[1]);  // h = 1
+    float a2 = __fadd_rn(r[2], r[3]), a3 = __fsub_rn(r[2], r[3]);
+    r[0] = __fadd_rn(a0, a2);  // h = 2
+    r[1] = __fadd_rn(a1, a3);
+    r[2] = __fsub_rn(a0, a2);
+    r[3] = __fsub_rn(a1, a3);
+#pragma unroll
+    for (int mask = 1; mask < 32; mask <<= 1) {  // h = 4 mask
+        const bool upper = (lane & mask) != 0;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            float other = __shfl_xor_sync(0xffffffffu, r[i], mask);
+            r[i] = upper ? __fsub_rn(other, r[i]) : __fadd_rn(r[i], other);
+        }
+    }
+}
+
+__device__ __forceinline__ float warp_max(float v) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+    return v;
+}
+
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    return v;
+}
+
+__device__ __forceinline__ int warp_sum_int(int v) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    return v;
+}
+
+// Statistics of one 128-element block (lane l holds elements 4l..4l+3):
+// {max |v|, max |H v|, sum v^2}.  Feeds the fused quantisation of a
+// consumer kernel, which recomputes H v with fwht128_warp bit for bit.
+__device__ __forceinline__ float3 block_stats128(float (&r)[4], int lane) {
+    float amax = fmaxf(fmaxf(fabsf(r[0]), fabsf(r[1])), fmaxf(fabsf(r[2]), fabsf(r[3])));
+    float ss = fmaf(r[3], r[3], fmaf(r[2], r[2], fmaf(r[1], r[1], r[0] * r[0])));
+    amax = warp_max(amax);
+    ss = warp_sum(ss);
+    fwht128_warp(r, lane);
+    float amaxh = fmaxf(fmaxf(fabsf(r[0]), fabsf(r[1])), fmaxf(fabsf(r[2]), fabsf(r[3])));
+    amaxh = warp_max(amaxh);
+    return make_float3(amax, amaxh, ss);
+}
+
+constexpr float kInvSqrt128 = 0.0883883476483184405501f;
+
 }  // namespace tern

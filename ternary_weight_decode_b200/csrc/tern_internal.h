@@ -57,8 +57,20 @@ struct GemvLaunch {
     const float *residual;
     void *out;  // y, h (fp32) or partials (int32)
     int ldo;
+    // fp32 input quantised inside the kernel (x != nullptr selects this form)
+    const float *x;
+    int ldx;
+    const float *x_stats;
+    int x_stats_ld;
+    int qflags;
+    // optional statistics of the output, per 128-row block
+    float *y_stats;
+    int y_stats_ld;
 };
 
 cudaError_t launch_gemv(const GemvLaunch &L, cudaStream_t s, const char **why);
+cudaError_t launch_act_stats(const float *x, int M, int K, int ldx, float *stats, int ld,
+                             cudaStream_t s);
+cudaError_t read_clear_device_error(int *value, cudaStream_t s);
 
 }  // namespace tern

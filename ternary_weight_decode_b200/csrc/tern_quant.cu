@@ -17,7 +17,6 @@
 namespace tern {
 
 constexpr int kQuantThreads = 512;
-constexpr float kInvSqrt128 = 0.0883883476483184405501f;
 
 template <bool FP16>
 __global__ void __launch_bounds__(kQuantThreads)
@@ -74,22 +73,8 @@ __global__ void __launch_bounds__(kQuantThreads)
         for (int b = warp; b < K / 128; b += nwarps) {
             float4 *p = reinterpret_cast<float4 *>(v + 128 * b + 4 * lane);
             float4 e = *p;
-            // h = 1: pairs (0,1), (2,3)
-            float a0 = __fadd_rn(e.x, e.y), a1 = __fsub_rn(e.x, e.y);
-            float a2 = __fadd_rn(e.z, e.w), a3 = __fsub_rn(e.z, e.w);
-            // h = 2: pairs (0,2), (1,3)
-            float r[4] = {__fadd_rn(a0, a2), __fadd_rn(a1, a3), __fsub_rn(a0, a2),
-                          __fsub_rn(a1, a3)};
-            // h = 4 .. 64: partner lane l ^ mask holds the element h away
-#pragma unroll
-            for (int mask = 1; mask < 32; mask <<= 1) {
-                const bool upper = (lane & mask) != 0;
-#pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    float other = __shfl_xor_sync(0xffffffffu, r[i], mask);
-                    r[i] = upper ? __fsub_rn(other, r[i]) : __fadd_rn(r[i], other);
-                }
-            }
+            float r[4] = {e.x, e.y, e.z, e.w};
+            fwht128_warp(r, lane);
             *p = make_float4(r[0], r[1], r[2], r[3]);
         }
         __syncthreads();

@@ -3,16 +3,18 @@ layer stack, run through the C ABI and replayed as one CUDA graph.
 
 The weight path of one decoder layer (Bonsai page, "Decode 为什么只能算一般":
 per layer the Q/K/V/O projections, then the Hadamard-rotated FFN input shared
-by the fused gate/up + SwiGLU kernel, then down; CUDA Graph replay):
+by the fused gate/up + SwiGLU kernel, then down; CUDA Graph replay).  Each
+projection quantises its own fp32 input inside the kernel, from the block
+statistics its producer wrote (4 launches per layer, 1 per step for the
+statistics of the step input):
 
-  1. act_quant_fwht(x)                  -> q1, s1        (K = 5120)
-  2. tern_gemv(Wqkv, q1)                -> qkv           (N = 7168 = q 5120 + k 1024 + v 1024)
-  3. act_quant_fwht(qkv[:, :5120])      -> q2, s2        (attention stand-in: the q output)
-  4. tern_gemv(Wo, q2, residual=x)      -> x             (N = 5120)
-  5. act_quant_fwht(x, Hadamard 128)    -> q3, s3
-  6. tern_gateup_swiglu(Wg, Wu, q3)     -> h             (N = 17408)
-  7. act_quant_fwht(h)                  -> q4, s4        (K = 17408)
-  8. tern_gemv(Wd, q4, residual=x)      -> x             (N = 5120)
+  1. tern_gemv_fused(Wqkv, x)                   -> qkv   (N = 7168 = q 5120 + k 1024 + v 1024)
+  2. tern_gemv_fused(Wo, qkv[:, :5120], +x)     -> x     (attention stand-in: the q output)
+  3. tern_gateup_swiglu_fused(Wg, Wu, H x)      -> h     (N = 17408, Hadamard-rotated input)
+  4. tern_gemv_fused(Wd, h, +x)                 -> x     (K = 17408)
+
+The unfused form (separate act_quant_fwht launches, 8 per layer) is kept as
+`fused=False` for comparison and for the int8-input entry points.
 
 Attention and norms are not on this path (the pages give no detail); the
 attention output is stood in by the q projection, and a weightless RMSNorm
@@ -68,6 +70,7 @@ class DecodeModel:
     hidden: int = HIDDEN
     qkv: int = QKV
     ffn: int = FFN
+    fused: bool = True
     layers: list = field(default_factory=list)
 
     def build(self, seed_base: int = 0):
@@ -93,13 +96,37 @@ class DecodeModel:
         self.q_h = torch.zeros((M, ld_h), dtype=torch.int8, device="cuda")
         self.q_f = torch.zeros((M, ld_f), dtype=torch.int8, device="cuda")
         self.s = torch.zeros((4, M), dtype=torch.float32, device="cuda")
+        self.st_x = tern.stats_buffer(M, self.hidden)
+        self.st_qkv = tern.stats_buffer(M, self.qkv)
+        self.st_x1 = tern.stats_buffer(M, self.hidden)
+        self.st_h = tern.stats_buffer(M, self.ffn)
         return self
 
     def bytes_per_step(self) -> int:
         return self.n_layers * layer_bytes(self.fmt, self.hidden, self.qkv, self.ffn)
 
     def launches_per_step(self) -> int:
-        return 8 * self.n_layers
+        return 4 * self.n_layers + 1 if self.fused else 8 * self.n_layers
+
+    def layer_step_fused(self, L: Layer, keep=None):
+        M = self.M
+        rms, rot = tern.TERN_QUANT_RMSNORM, tern.TERN_QUANT_FWHT128
+        if keep is not None:
+            keep.append(("qkv_in", self.x.clone()))
+        tern.tern_gemv_fused(L.wqkv, self.x, self.st_x, self.qkv_out, qflags=rms,
+                             y_stats=self.st_qkv, M=M)
+        if keep is not None:
+            keep.append(("o_in", self.qkv_out.clone(), self.x.clone()))
+        tern.tern_gemv_fused(L.wo, self.qkv_out[:, : self.hidden], self.st_qkv, self.x, qflags=rms,
+                             residual=self.x, y_stats=self.st_x1, M=M)
+        if keep is not None:
+            keep.append(("ffn_in", self.x.clone()))
+        tern.tern_gateup_swiglu_fused(L.wg, L.wu, self.x, self.st_x1, self.h, qflags=rms | rot,
+                                      h_stats=self.st_h, M=M)
+        if keep is not None:
+            keep.append(("down_in", self.h.clone(), self.x.clone()))
+        tern.tern_gemv_fused(L.wd, self.h, self.st_h, self.x, qflags=rms, residual=self.x,
+                             y_stats=self.st_x, M=M)
 
     def layer_step(self, L: Layer, keep=None):
         M = self.M
@@ -119,9 +146,14 @@ class DecodeModel:
             keep.append(("down_in", self.q_f.clone(), self.s[3].clone(), self.x.clone(), self.h.clone()))
         tern.tern_gemv(L.wd, self.q_f, self.s[3], self.x, residual=self.x, M=M)
 
-    def step(self):
-        for L in self.layers:
-            self.layer_step(L)
+    def step(self, keep=None):
+        if self.fused:
+            tern.tern_act_stats(self.x, self.st_x)
+            for L in self.layers:
+                self.layer_step_fused(L, keep)
+        else:
+            for L in self.layers:
+                self.layer_step(L, keep)
 
     def capture(self) -> torch.cuda.CUDAGraph:
         """One CUDA graph holding the whole step (8 launches per layer)."""

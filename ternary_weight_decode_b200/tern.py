@@ -22,6 +22,7 @@ TERN_OK, TERN_EINVAL, TERN_ECUDA, TERN_EUNSUPPORTED, TERN_ETIMEOUT = 0, 1, 2, 3,
 TERN_FMT_BASE3, TERN_FMT_2BIT = 0, 1
 TERN_MATRIX_STATIC = 1
 TERN_QUANT_RMSNORM = 1
+TERN_QUANT_FWHT128 = 2
 GROUP = 128
 
 
@@ -76,6 +77,10 @@ def lib() -> ctypes.CDLL:
                 "tern_gateup_swiglu": (ctypes.c_int, [pm, pm, p, i32, p, i32, p, i32, p]),
                 "tern_debug_group_partials": (ctypes.c_int, [pm, p, i32, i32, p, p]),
                 "tern_device_error": (ctypes.c_int, [ctypes.POINTER(i32), p]),
+                "tern_act_stats": (ctypes.c_int, [p, i32, i32, i32, p, i32, p]),
+                "tern_gemv_fused": (ctypes.c_int, [pm, p, i32, p, i32, i32, i32, p, p, i32, p, i32, p]),
+                "tern_gateup_swiglu_fused": (ctypes.c_int, [pm, pm, p, i32, p, i32, i32, i32, p, i32,
+                                                            p, i32, p]),
             }
             for name, (res, args) in sig.items():
                 f = getattr(L, name)
@@ -220,6 +225,48 @@ def tern_debug_group_partials(W: TernMatrix, q: torch.Tensor, P: torch.Tensor,
     s = W.struct()
     _check(lib().tern_debug_group_partials(ctypes.byref(s), _ptr(q), q.stride(0), M, _ptr(P),
                                            _stream(stream)), "tern_debug_group_partials")
+
+
+def stats_buffer(M: int, length: int, device="cuda") -> torch.Tensor:
+    """A statistics buffer fp32 [M, ceil(length/128), 4] for the fused calls."""
+    return torch.zeros((M, (length + 127) // 128, 4), dtype=torch.float32, device=device)
+
+
+def tern_act_stats(x: torch.Tensor, stats: torch.Tensor, K: int | None = None, stream=None):
+    assert x.dtype == torch.float32 and x.stride(1) == 1 and stats.dtype == torch.float32
+    M = x.shape[0]
+    K = x.shape[1] if K is None else K
+    _check(lib().tern_act_stats(_ptr(x), M, K, x.stride(0), _ptr(stats), stats.shape[1],
+                                _stream(stream)), "tern_act_stats")
+
+
+def tern_gemv_fused(W: TernMatrix, x: torch.Tensor, x_stats: torch.Tensor, y: torch.Tensor,
+                    qflags: int = 0, residual: torch.Tensor | None = None,
+                    y_stats: torch.Tensor | None = None, M: int | None = None, stream=None):
+    """y = [residual +] W . quant(x); x fp32 [M, >=K] with block statistics x_stats."""
+    M = x.shape[0] if M is None else M
+    assert x.dtype == torch.float32 and x.stride(1) == 1 and y.dtype == torch.float32
+    if residual is not None:
+        assert residual.dtype == torch.float32 and residual.stride(0) == y.stride(0)
+    s = W.struct()
+    _check(lib().tern_gemv_fused(ctypes.byref(s), _ptr(x), x.stride(0), _ptr(x_stats),
+                                 x_stats.shape[1], qflags, M, _ptr(residual), _ptr(y), y.stride(0),
+                                 _ptr(y_stats), 0 if y_stats is None else y_stats.shape[1],
+                                 _stream(stream)), "tern_gemv_fused")
+
+
+def tern_gateup_swiglu_fused(Wg: TernMatrix, Wu: TernMatrix, x: torch.Tensor,
+                             x_stats: torch.Tensor, h: torch.Tensor, qflags: int = 0,
+                             h_stats: torch.Tensor | None = None, M: int | None = None,
+                             stream=None):
+    M = x.shape[0] if M is None else M
+    assert x.dtype == torch.float32 and x.stride(1) == 1 and h.dtype == torch.float32
+    sg, su = Wg.struct(), Wu.struct()
+    _check(lib().tern_gateup_swiglu_fused(ctypes.byref(sg), ctypes.byref(su), _ptr(x), x.stride(0),
+                                          _ptr(x_stats), x_stats.shape[1], qflags, M, _ptr(h),
+                                          h.stride(0), _ptr(h_stats),
+                                          0 if h_stats is None else h_stats.shape[1],
+                                          _stream(stream)), "tern_gateup_swiglu_fused")
 
 
 def tern_device_error(stream=None) -> int:
