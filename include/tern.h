@@ -239,6 +239,28 @@ tern_status tern_gateup_swiglu_fused(const tern_matrix *Wg, const tern_matrix *W
                                      int32_t h_stats_ld, void *stream);
 
 /*
+ * Test hook for the tensor-core path (no counterpart on the pages; it pins
+ * the tcgen05 encodings the kernels use): one CTA computes
+ *   D[m][n] = sum_k A[m][k] * B[n][k]   (int32, exact)
+ * for A int8 [128][K] (row-major; read as unsigned bytes when a_signed == 0)
+ * and B int8 [N][K] (row-major; unsigned when b_signed == 0), with A taken
+ * from tensor memory (a_in_smem == 0) or shared memory (1).
+ * K in 32..512, a multiple of 32; N in 16..256, a multiple of 16.
+ * A, B: device, 16-byte aligned; D: device int32 [128][N].
+ */
+tern_status tern_debug_mma_i8(int32_t a_in_smem, const int8_t *A, int32_t a_signed,
+                              const int8_t *B, int32_t b_signed, int32_t *D,
+                              int32_t K, int32_t N, void *stream);
+
+/*
+ * Test hook: selects the engine of the GEMV entry points for the calling
+ * process -- 0: tensor cores (tcgen05), 1: CUDA cores (dp4a, the default).
+ * Both compute the same integers; the tests compare them.
+ * tern_debug_group_partials always uses the CUDA-core engine.
+ */
+tern_status tern_debug_select_engine(int32_t engine);
+
+/*
  * Reads and clears the device error word of the current device: 0 when no
  * bounded wait in a kernel ran out since the last call, else a nonzero code.
  * Synchronises `stream`.

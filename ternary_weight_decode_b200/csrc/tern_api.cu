@@ -276,6 +276,23 @@ tern_status tern_act_stats(const float *x, int32_t M, int32_t K, int32_t ldx, fl
                        "tern_act_stats");
 }
 
+tern_status tern_debug_mma_i8(int32_t a_in_smem, const int8_t *A, int32_t a_signed, const int8_t *B,
+                              int32_t b_signed, int32_t *D, int32_t K, int32_t N, void *stream) {
+    if (K < 32 || K > 512 || K % 32 != 0) return fail(TERN_EINVAL, "tern_debug_mma_i8: K must be 32..512, a multiple of 32%s");
+    if (N < 16 || N > 256 || N % 16 != 0) return fail(TERN_EINVAL, "tern_debug_mma_i8: N must be 16..256, a multiple of 16%s");
+    if (!A || !B || !D || !aligned(A, 16) || !aligned(B, 16) || !aligned(D, 16))
+        return fail(TERN_EINVAL, "tern_debug_mma_i8: pointers must be 16-byte aligned%s");
+    return cuda_status(tern::launch_debug_mma(a_in_smem ? 1 : 0, A, a_signed ? 1 : 0, B, b_signed ? 1 : 0,
+                                              D, K, N, static_cast<cudaStream_t>(stream)),
+                       "tern_debug_mma_i8");
+}
+
+tern_status tern_debug_select_engine(int32_t engine) {
+    if (engine != 0 && engine != 1) return fail(TERN_EINVAL, "tern_debug_select_engine: engine must be 0 or 1%s");
+    tern::select_engine(engine);
+    return TERN_OK;
+}
+
 static tern_status check_fused_input(const float *x, int32_t ldx, int32_t K, const float *x_stats,
                                      int32_t x_stats_ld, int32_t qflags, int32_t M) {
     if (M < 1 || M > 16) return fail(TERN_EINVAL, "fused: M must be in 1..16%s");

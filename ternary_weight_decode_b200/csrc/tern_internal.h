@@ -69,8 +69,14 @@ struct GemvLaunch {
 };
 
 cudaError_t launch_gemv(const GemvLaunch &L, cudaStream_t s, const char **why);
+cudaError_t launch_gemv_tc(const GemvLaunch &L, cudaStream_t s, const char **why);
+void select_engine(int engine);  // 0: tensor cores, 1: CUDA cores (default)
 cudaError_t launch_act_stats(const float *x, int M, int K, int ldx, float *stats, int ld,
                              cudaStream_t s);
 cudaError_t read_clear_device_error(int *value, cudaStream_t s);
+
+// ---------------------------------------------------------------- tcgen05 test hook
+cudaError_t launch_debug_mma(int a_in_smem, const int8_t *A, int a_signed, const int8_t *B,
+                             int b_signed, int32_t *D, int K, int N, cudaStream_t s);
 
 }  // namespace tern

@@ -78,6 +78,8 @@ def lib() -> ctypes.CDLL:
                 "tern_debug_group_partials": (ctypes.c_int, [pm, p, i32, i32, p, p]),
                 "tern_device_error": (ctypes.c_int, [ctypes.POINTER(i32), p]),
                 "tern_act_stats": (ctypes.c_int, [p, i32, i32, i32, p, i32, p]),
+                "tern_debug_mma_i8": (ctypes.c_int, [i32, p, i32, p, i32, p, i32, i32, p]),
+                "tern_debug_select_engine": (ctypes.c_int, [i32]),
                 "tern_gemv_fused": (ctypes.c_int, [pm, p, i32, p, i32, i32, i32, p, p, i32, p, i32, p]),
                 "tern_gateup_swiglu_fused": (ctypes.c_int, [pm, pm, p, i32, p, i32, i32, i32, p, i32,
                                                             p, i32, p]),
@@ -267,6 +269,24 @@ def tern_gateup_swiglu_fused(Wg: TernMatrix, Wu: TernMatrix, x: torch.Tensor,
                                           h.stride(0), _ptr(h_stats),
                                           0 if h_stats is None else h_stats.shape[1],
                                           _stream(stream)), "tern_gateup_swiglu_fused")
+
+
+def tern_debug_mma_i8(A: torch.Tensor, B: torch.Tensor, D: torch.Tensor, a_in_smem: bool = False,
+                      a_signed: bool = True, b_signed: bool = True, stream=None):
+    """D int32 [128, N] = A [128, K] . B [N, K]^T on the tensor cores (test hook)."""
+    K = A.shape[1]
+    N = B.shape[0]
+    _check(lib().tern_debug_mma_i8(1 if a_in_smem else 0, _ptr(A), 1 if a_signed else 0, _ptr(B),
+                                   1 if b_signed else 0, _ptr(D), K, N, _stream(stream)),
+           "tern_debug_mma_i8")
+
+
+ENGINE_TENSOR_CORES, ENGINE_CUDA_CORES = 0, 1
+
+
+def tern_debug_select_engine(engine: int):
+    """Test hook: 0 = tensor-core GEMV engine, 1 = CUDA-core engine (default)."""
+    _check(lib().tern_debug_select_engine(engine), "tern_debug_select_engine")
 
 
 def tern_device_error(stream=None) -> int:
