@@ -43,6 +43,8 @@ def parse():
     ap.add_argument("--fmt", choices=["base3", "2bit"], default="base3")
     ap.add_argument("--layers", type=int, default=64)
     ap.add_argument("--M", type=int, default=1)
+    ap.add_argument("--mode", choices=["auto", "streamed", "fused", "unfused"], default="auto",
+                    help="decode-step kernels (auto: streamed for M <= 2, else fused)")
     ap.add_argument("--cpu-seconds", type=float, default=10.0,
                     help="target CPU time of the oracle baseline sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -247,6 +249,7 @@ def workload_config(args):
                         if args.layers == 64 else
                         f"{args.layers}-layer 27B-shape ternary decode stream ({args.fmt}), batch {args.M}",
             "layers": args.layers, "format": args.fmt, "batch": args.M,
+            "kernels": args.mode if args.mode != "auto" else ("streamed" if args.M <= 2 else "fused"),
             "l2": "inputs larger than L2: each step streams every layer's weights once"}
 
 
@@ -267,7 +270,8 @@ def main():
 
     torch.cuda.set_device(local)
     fmt_id = tern.TERN_FMT_BASE3 if args.fmt == "base3" else tern.TERN_FMT_2BIT
-    model = decode.DecodeModel(fmt_id, args.layers, M=args.M).build(seed_base=0)
+    mode = args.mode if args.mode != "auto" else ("streamed" if args.M <= 2 else "fused")
+    model = decode.DecodeModel(fmt_id, args.layers, M=args.M, mode=mode).build(seed_base=0)
     x0 = torch.from_numpy(synth.activations(0, args.M, decode.HIDDEN).astype(np.float32))
     x0_host = x0.pin_memory()
     out_host = torch.empty_like(x0_host).pin_memory()
@@ -284,8 +288,18 @@ def main():
     gu_bytes = 2 * (decode.FFN * tern.tern_canonical_row_bytes(fmt_id, decode.HIDDEN)
                     + 2 * decode.FFN * (decode.HIDDEN // 128))
     def gateup_all():
+        rms, rot = tern.TERN_QUANT_RMSNORM, tern.TERN_QUANT_FWHT128
         for L in model.layers:
-            tern.tern_gateup_swiglu(L.wg, L.wu, model.q_h, model.s[2], model.h, M=args.M)
+            if mode == "streamed":
+                tern.tern_gateup_swiglu_streamed(L.wg, L.wu, model.x, model.h, model.ws,
+                                                 qflags=rms | rot, M=args.M)
+            elif mode == "fused":
+                tern.tern_gateup_swiglu_fused(L.wg, L.wu, model.x, model.st_x1, model.h,
+                                              qflags=rms | rot, M=args.M)
+            else:
+                tern.tern_gateup_swiglu(L.wg, L.wu, model.q_h, model.s[2], model.h, M=args.M)
+    if mode == "fused":
+        tern.tern_act_stats(model.x, model.st_x1)
     gateup_all()
     torch.cuda.synchronize()
     gu_graph = torch.cuda.CUDAGraph()

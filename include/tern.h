@@ -90,9 +90,26 @@ typedef struct tern_matrix {
                               >= the used row bytes */
     const void *packed;    /* device, 16-byte aligned, N * row_stride bytes */
     const uint16_t *scales;/* device, 2-byte aligned, N * ceil(K/group) fp16 */
+    const uint16_t *scales_tiled; /* optional, device, 16-byte aligned: the same
+                              scales re-tiled by tern_retile_scales; required
+                              by the streamed entry points, else may be NULL */
     int32_t flags;         /* TERN_MATRIX_STATIC or 0 */
     int32_t reserved;      /* must be 0 */
 } tern_matrix;
+
+/*
+ * Load-time re-tile of the group scales into the order the streamed kernels
+ * consume them (Bonsai page, "后面还有没有优化空间": re-tile codes and
+ * scales at load time).  A "unit" is 32 rows x one 128-byte superblock of
+ * codes (640 positions = 5 groups in TERN_FMT_BASE3, 512 = 4 groups in
+ * TERN_FMT_2BIT); units are numbered rb * SB + sb with rb = row / 32 and SB =
+ * ceil(used row bytes / 128).  Unit u holds 32 rows x GPS fp16 scales
+ * (GPS = 5 or 4), row-major, zero past N and past ceil(K/128):
+ *   out[(u * 32 + r) * GPS + g] = scales[(32 rb + r) * G + GPS sb + g].
+ * out: device, 16-byte aligned, tern_tiled_scales_bytes() bytes.
+ */
+tern_status tern_tiled_scales_bytes(int32_t fmt, int32_t N, int32_t K, size_t *bytes);
+tern_status tern_retile_scales(const tern_matrix *W, uint16_t *out, void *stream);
 
 /* Human-readable name of a status code (static storage). */
 const char *tern_status_string(tern_status s);
@@ -237,6 +254,36 @@ tern_status tern_gateup_swiglu_fused(const tern_matrix *Wg, const tern_matrix *W
                                      int32_t qflags, int32_t M, float *h,
                                      int32_t ldh, float *h_stats,
                                      int32_t h_stats_ld, void *stream);
+
+/*
+ * Streamed forms of tern_gemv_fused / tern_gateup_swiglu_fused for decode
+ * with M = 1 or 2 token rows, same results and arguments apart from these:
+ *  - the activation statistics are not needed: every CTA forms the row
+ *    scale from x itself (max |x|, or max |H x| with TERN_QUANT_FWHT128);
+ *  - W->scales_tiled must hold the re-tiled scales (tern_retile_scales);
+ *  - workspace: device, 16-byte aligned, >= tern_stream_workspace_bytes()
+ *    bytes, all zero before its first use.  It holds fp32 partial sums
+ *    (scratch) from its start and one int32 arrival counter per 32-row
+ *    block from its end backwards (block rb at byte ws_bytes - 4 (rb + 1),
+ *    ws_bytes rounded down to a multiple of 4); every call leaves the
+ *    counters zero again, so one workspace, sized for the largest call,
+ *    serves a whole chain of calls of any sizes on one stream (calls that
+ *    may overlap need separate workspaces).
+ * One CTA per SM streams an equal share of the matrix's 32-row x 128-byte
+ * tiles; with TERN_MATRIX_STATIC the tiles start streaming before the
+ * previous kernel on the stream has finished.  x must not overlap y / h.
+ */
+tern_status tern_stream_workspace_bytes(int32_t fmt, int32_t N, int32_t M,
+                                        int32_t two_matrices, size_t *bytes);
+tern_status tern_gemv_streamed(const tern_matrix *W, const float *x, int32_t ldx,
+                               int32_t qflags, int32_t M, const float *residual,
+                               float *y, int32_t ldy, void *workspace,
+                               size_t ws_bytes, void *stream);
+tern_status tern_gateup_swiglu_streamed(const tern_matrix *Wg, const tern_matrix *Wu,
+                                        const float *x, int32_t ldx, int32_t qflags,
+                                        int32_t M, float *h, int32_t ldh,
+                                        void *workspace, size_t ws_bytes,
+                                        void *stream);
 
 /*
  * Test hook for the tensor-core path (no counterpart on the pages; it pins

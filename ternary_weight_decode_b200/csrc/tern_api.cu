@@ -38,6 +38,8 @@ tern_status check_matrix(const tern_matrix *W, const char *name) {
         return fail(TERN_EINVAL, "%s: packed must be a 16-byte aligned device pointer", name);
     if (!W->scales || !aligned(W->scales, 2))
         return fail(TERN_EINVAL, "%s: scales must be a 2-byte aligned device pointer", name);
+    if (W->scales_tiled && !aligned(W->scales_tiled, 16))
+        return fail(TERN_EINVAL, "%s: scales_tiled must be 16-byte aligned", name);
     if (W->flags & ~TERN_MATRIX_STATIC) return fail(TERN_EINVAL, "%s: unknown flag bits", name);
     if (W->reserved != 0) return fail(TERN_EINVAL, "%s: reserved must be 0", name);
     return TERN_OK;
@@ -86,6 +88,22 @@ tern_status tern_canonical_row_bytes(int32_t fmt, int32_t K, int64_t *bytes) {
     if (K < 1 || !bytes) return fail(TERN_EINVAL, "K must be >= 1 and bytes non-null%s");
     *bytes = tern::canonical_row_bytes(fmt, K);
     return TERN_OK;
+}
+
+tern_status tern_tiled_scales_bytes(int32_t fmt, int32_t N, int32_t K, size_t *bytes) {
+    if (!valid_fmt(fmt)) return fail(TERN_EINVAL, "tern_tiled_scales_bytes: unknown format%s");
+    if (N < 1 || K < 1 || !bytes) return fail(TERN_EINVAL, "tern_tiled_scales_bytes: bad arguments%s");
+    *bytes = static_cast<size_t>(tern::tiled_scales_bytes(fmt, N, K));
+    return TERN_OK;
+}
+
+tern_status tern_retile_scales(const tern_matrix *W, uint16_t *out, void *stream) {
+    tern_status st = check_matrix(W, "tern_retile_scales");
+    if (st != TERN_OK) return st;
+    if (!out || !aligned(out, 16)) return fail(TERN_EINVAL, "tern_retile_scales: out must be 16-byte aligned%s");
+    return cuda_status(tern::launch_retile_scales(W->fmt, W->scales, W->N, W->K, out,
+                                                  static_cast<cudaStream_t>(stream)),
+                       "tern_retile_scales");
 }
 
 tern_status tern_pack(int32_t fmt, const int8_t *trits, int32_t N, int32_t K, void *packed_out,
@@ -285,6 +303,87 @@ tern_status tern_debug_mma_i8(int32_t a_in_smem, const int8_t *A, int32_t a_sign
     return cuda_status(tern::launch_debug_mma(a_in_smem ? 1 : 0, A, a_signed ? 1 : 0, B, b_signed ? 1 : 0,
                                               D, K, N, static_cast<cudaStream_t>(stream)),
                        "tern_debug_mma_i8");
+}
+
+tern_status tern_stream_workspace_bytes(int32_t fmt, int32_t N, int32_t M, int32_t two_matrices,
+                                        size_t *bytes) {
+    if (!valid_fmt(fmt) || N < 1 || M < 1 || M > 2 || !bytes)
+        return fail(TERN_EINVAL, "tern_stream_workspace_bytes: bad arguments (M must be 1 or 2)%s");
+    *bytes = tern::stream_workspace_bytes(fmt, N, M, two_matrices ? 2 : 1);
+    return TERN_OK;
+}
+
+static tern_status run_streamed(const tern_matrix *W0, const tern_matrix *W1, const float *x,
+                                int32_t ldx, int32_t qflags, int32_t M, const float *residual,
+                                float *out, int32_t ldo, void *workspace, size_t ws_bytes,
+                                void *stream, const char *name) {
+    if (M < 1 || M > 2) return fail(TERN_EUNSUPPORTED, "%s: the streamed kernels take M = 1 or 2", name);
+    if (!W0->scales_tiled || (W1 && !W1->scales_tiled))
+        return fail(TERN_EINVAL, "%s: scales_tiled is required (tern_retile_scales)", name);
+    if (!x || !aligned(x, 16) || ldx < W0->K || ldx % 4 != 0)
+        return fail(TERN_EINVAL, "%s: x must be 16-byte aligned, ldx >= K, ldx %% 4 == 0", name);
+    if (qflags & ~(TERN_QUANT_FWHT128 | TERN_QUANT_RMSNORM)) return fail(TERN_EINVAL, "%s: unknown qflags", name);
+    if ((qflags & TERN_QUANT_FWHT128) && W0->K % 128 != 0)
+        return fail(TERN_EINVAL, "%s: the Hadamard rotation needs K %% 128 == 0", name);
+    if (!out || !aligned(out, 4) || ldo < W0->N) return fail(TERN_EINVAL, "%s: bad output or its stride", name);
+    if (residual && !aligned(residual, 4)) return fail(TERN_EINVAL, "%s: bad residual", name);
+    const size_t need = tern::stream_workspace_bytes(W0->fmt, W0->N, M, W1 ? 2 : 1);
+    if (!workspace || !aligned(workspace, 16) || ws_bytes < need)
+        return fail(TERN_EINVAL, "%s: workspace missing, misaligned or too small", name);
+    int dev = 0, sms = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (e != cudaSuccess) return cuda_status(e, name);
+    tern::StreamLaunch S = {};
+    S.fmt = W0->fmt;
+    S.swiglu = W1 ? 1 : 0;
+    S.N = W0->N;
+    S.K = W0->K;
+    S.row_bytes = tern::device_row_bytes(W0->fmt, W0->K);
+    S.row_stride = W0->row_stride;
+    S.packed[0] = W0->packed;
+    S.packed[1] = W1 ? W1->packed : W0->packed;
+    S.scales_tiled[0] = W0->scales_tiled;
+    S.scales_tiled[1] = W1 ? W1->scales_tiled : W0->scales_tiled;
+    S.prefetch_ok = ((W0->flags & (W1 ? W1->flags : W0->flags)) & TERN_MATRIX_STATIC) ? 1 : 0;
+    S.x = x;
+    S.ldx = ldx;
+    S.qflags = qflags;
+    S.M = M;
+    S.residual = residual;
+    S.out = out;
+    S.ldo = ldo;
+    S.workspace = workspace;
+    S.ws_bytes = ws_bytes;
+    S.num_sms = sms;
+    const char *why = nullptr;
+    e = tern::launch_gemv_stream(S, static_cast<cudaStream_t>(stream), &why);
+    if (why) return fail(TERN_EUNSUPPORTED, "%s", why);
+    return cuda_status(e, name);
+}
+
+tern_status tern_gemv_streamed(const tern_matrix *W, const float *x, int32_t ldx, int32_t qflags,
+                               int32_t M, const float *residual, float *y, int32_t ldy,
+                               void *workspace, size_t ws_bytes, void *stream) {
+    tern_status st = check_matrix(W, "tern_gemv_streamed");
+    if (st != TERN_OK) return st;
+    return run_streamed(W, nullptr, x, ldx, qflags, M, residual, y, ldy, workspace, ws_bytes, stream,
+                        "tern_gemv_streamed");
+}
+
+tern_status tern_gateup_swiglu_streamed(const tern_matrix *Wg, const tern_matrix *Wu, const float *x,
+                                        int32_t ldx, int32_t qflags, int32_t M, float *h,
+                                        int32_t ldh, void *workspace, size_t ws_bytes,
+                                        void *stream) {
+    tern_status st = check_matrix(Wg, "tern_gateup_swiglu_streamed (gate)");
+    if (st != TERN_OK) return st;
+    st = check_matrix(Wu, "tern_gateup_swiglu_streamed (up)");
+    if (st != TERN_OK) return st;
+    if (Wg->fmt != Wu->fmt || Wg->N != Wu->N || Wg->K != Wu->K || Wg->group != Wu->group ||
+        Wg->row_stride != Wu->row_stride)
+        return fail(TERN_EINVAL, "tern_gateup_swiglu_streamed: gate and up must share fmt, N, K, group, row_stride%s");
+    return run_streamed(Wg, Wu, x, ldx, qflags, M, nullptr, h, ldh, workspace, ws_bytes, stream,
+                        "tern_gateup_swiglu_streamed");
 }
 
 tern_status tern_debug_select_engine(int32_t engine) {

@@ -169,6 +169,11 @@ __device__ __forceinline__ void fwht128_warp(float (&r)[4], int lane) {
     }
 }
 
+// Named barrier over `count` threads (a multiple of 32; id 0 is __syncthreads).
+__device__ __forceinline__ void warpgroup_sync_n(int id, int count) {
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
+
 __device__ __forceinline__ float warp_max(float v) {
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));

@@ -212,6 +212,21 @@ __global__ void export_kernel(int fmt, const uint8_t *__restrict__ packed, int N
     if (bad && d_invalid) atomicAdd(d_invalid, bad);
 }
 
+// Unit-major scales: unit u = rb * SB + sb holds 32 rows x gps scales.
+__global__ void retile_scales_kernel(const uint16_t *__restrict__ sc, int N, int G, int SB, int gps,
+                                     int64_t units, uint16_t *__restrict__ out) {
+    const int64_t total = units * 32 * gps;
+    for (int64_t idx = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; idx < total;
+         idx += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+        const int64_t u = idx / (32 * gps);
+        const int r = static_cast<int>((idx / gps) % 32);
+        const int g = static_cast<int>(idx % gps);
+        const int64_t rb = u / SB, sb = u % SB;
+        const int64_t n = rb * 32 + r, gg = sb * gps + g;
+        out[idx] = (n < N && gg < G) ? sc[n * G + gg] : static_cast<uint16_t>(0);
+    }
+}
+
 static int grid_for(int64_t total) {
     int64_t blocks = (total + 255) / 256;
     if (blocks < 1) blocks = 1;
@@ -241,6 +256,16 @@ cudaError_t launch_import(int fmt, const uint8_t *canon, int N, int K, void *out
     int64_t cbytes = canonical_row_bytes(fmt, K);
     import_kernel<<<grid_for(static_cast<int64_t>(N) * row_stride), 256, 0, s>>>(
         fmt, canon, N, K, cbytes, static_cast<uint8_t *>(out), row_stride, used, d_invalid);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_retile_scales(int fmt, const uint16_t *sc, int N, int K, uint16_t *out,
+                                 cudaStream_t s) {
+    const int G = static_cast<int>(ceil_div(K, 128));
+    const int SB = static_cast<int>(ceil_div(device_row_bytes(fmt, K), 128));
+    const int gps = (fmt == TERN_FMT_BASE3) ? 5 : 4;
+    const int64_t units = ceil_div(N, 32) * SB;
+    retile_scales_kernel<<<grid_for(units * 32 * gps), 256, 0, s>>>(sc, N, G, SB, gps, units, out);
     return cudaGetLastError();
 }
 

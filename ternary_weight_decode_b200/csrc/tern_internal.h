@@ -10,6 +10,8 @@
 
 namespace tern {
 
+inline int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
+
 inline int64_t device_row_bytes(int fmt, int64_t K) {
     if (fmt == TERN_FMT_BASE3) return 4 * ((K + 19) / 20);
     if (fmt == TERN_FMT_2BIT) return 4 * ((K + 15) / 16);
@@ -22,8 +24,6 @@ inline int64_t canonical_row_bytes(int fmt, int64_t K) {
     return -1;
 }
 
-inline int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
-
 // ---------------------------------------------------------------- format
 cudaError_t launch_pack(int fmt, const int8_t *trits, int N, int K, void *out, int64_t row_stride,
                         int32_t *d_invalid, cudaStream_t s);
@@ -33,6 +33,14 @@ cudaError_t launch_import(int fmt, const uint8_t *canon, int N, int K, void *out
                           int64_t row_stride, int32_t *d_invalid, cudaStream_t s);
 cudaError_t launch_export(int fmt, const void *packed, int N, int K, int64_t row_stride,
                           uint8_t *canon, int32_t *d_invalid, cudaStream_t s);
+cudaError_t launch_retile_scales(int fmt, const uint16_t *sc, int N, int K, uint16_t *out,
+                                 cudaStream_t s);
+
+inline int64_t tiled_scales_bytes(int fmt, int64_t N, int64_t K) {
+    const int64_t SB = ceil_div(device_row_bytes(fmt, K), 128);
+    const int64_t gps = (fmt == TERN_FMT_BASE3) ? 5 : 4;
+    return ceil_div(N, 32) * SB * 32 * gps * 2;
+}
 
 // ---------------------------------------------------------------- quant
 cudaError_t launch_act_quant(const void *x, bool fp16, int M, int K, int ldx, int fwht_block,
@@ -69,6 +77,26 @@ struct GemvLaunch {
 };
 
 cudaError_t launch_gemv(const GemvLaunch &L, cudaStream_t s, const char **why);
+
+// Streamed (persistent, evenly split) GEMV of tern_gemv_stream.cu.
+struct StreamLaunch {
+    int fmt, swiglu;
+    int N, K;
+    int64_t row_bytes, row_stride;
+    const void *packed[2];
+    const uint16_t *scales_tiled[2];
+    int prefetch_ok;
+    const float *x;
+    int ldx, qflags, M;
+    const float *residual;
+    float *out;
+    int ldo;
+    void *workspace;
+    size_t ws_bytes;
+    int num_sms;
+};
+size_t stream_workspace_bytes(int fmt, int N, int M, int nmat);
+cudaError_t launch_gemv_stream(const StreamLaunch &S, cudaStream_t s, const char **why);
 cudaError_t launch_gemv_tc(const GemvLaunch &L, cudaStream_t s, const char **why);
 void select_engine(int engine);  // 0: tensor cores, 1: CUDA cores (default)
 cudaError_t launch_act_stats(const float *x, int M, int K, int ldx, float *stats, int ld,

@@ -13,8 +13,11 @@ statistics of the step input):
   3. tern_gateup_swiglu_fused(Wg, Wu, H x)      -> h     (N = 17408, Hadamard-rotated input)
   4. tern_gemv_fused(Wd, h, +x)                 -> x     (K = 17408)
 
-The unfused form (separate act_quant_fwht launches, 8 per layer) is kept as
-`fused=False` for comparison and for the int8-input entry points.
+By default (M = 1 or 2) the projections run as the streamed kernels, which
+need no statistics (each CTA quantises the input itself) and split every
+matrix evenly over the SMs.  The fused form with statistics ("fused") and
+the unfused form with separate act_quant_fwht launches ("unfused", 8 per
+layer) are kept for comparison and for M > 2.
 
 Attention and norms are not on this path (the pages give no detail); the
 attention output is stood in by the q projection, and a weightless RMSNorm
@@ -70,8 +73,12 @@ class DecodeModel:
     hidden: int = HIDDEN
     qkv: int = QKV
     ffn: int = FFN
-    fused: bool = True
+    mode: str = "streamed"  # "streamed" (M <= 2), "fused" or "unfused"
     layers: list = field(default_factory=list)
+
+    @property
+    def fused(self) -> bool:
+        return self.mode != "unfused"
 
     def build(self, seed_base: int = 0):
         scratch = torch.empty(max(self.qkv, self.ffn) * max(self.hidden, self.ffn),
@@ -86,6 +93,12 @@ class DecodeModel:
                 make_matrix(self.fmt, self.hidden, self.ffn, s, synth.stream_id(l, synth.PROJ_DOWN), scratch),
             ))
         del scratch
+        if self.mode == "streamed":
+            assert self.M <= 2, "the streamed kernels take M = 1 or 2"
+            for L in self.layers:
+                for W in (L.wqkv, L.wo, L.wg, L.wu, L.wd):
+                    W.retile_scales()
+            self.ws = tern.stream_workspace(self.fmt, max(self.qkv, self.ffn, self.hidden), self.M, True)
         torch.cuda.synchronize()
         M = self.M
         ld_h = ((self.hidden + 15) // 16) * 16
@@ -106,7 +119,26 @@ class DecodeModel:
         return self.n_layers * layer_bytes(self.fmt, self.hidden, self.qkv, self.ffn)
 
     def launches_per_step(self) -> int:
-        return 4 * self.n_layers + 1 if self.fused else 8 * self.n_layers
+        if self.mode == "streamed":
+            return 4 * self.n_layers
+        return 4 * self.n_layers + 1 if self.mode == "fused" else 8 * self.n_layers
+
+    def layer_step_streamed(self, L: Layer, keep=None):
+        M = self.M
+        rms, rot = tern.TERN_QUANT_RMSNORM, tern.TERN_QUANT_FWHT128
+        if keep is not None:
+            keep.append(("qkv_in", self.x.clone()))
+        tern.tern_gemv_streamed(L.wqkv, self.x, self.qkv_out, self.ws, qflags=rms, M=M)
+        if keep is not None:
+            keep.append(("o_in", self.qkv_out.clone(), self.x.clone()))
+        tern.tern_gemv_streamed(L.wo, self.qkv_out[:, : self.hidden], self.x, self.ws, qflags=rms,
+                                residual=self.x, M=M)
+        if keep is not None:
+            keep.append(("ffn_in", self.x.clone()))
+        tern.tern_gateup_swiglu_streamed(L.wg, L.wu, self.x, self.h, self.ws, qflags=rms | rot, M=M)
+        if keep is not None:
+            keep.append(("down_in", self.h.clone(), self.x.clone()))
+        tern.tern_gemv_streamed(L.wd, self.h, self.x, self.ws, qflags=rms, residual=self.x, M=M)
 
     def layer_step_fused(self, L: Layer, keep=None):
         M = self.M
@@ -147,7 +179,10 @@ class DecodeModel:
         tern.tern_gemv(L.wd, self.q_f, self.s[3], self.x, residual=self.x, M=M)
 
     def step(self, keep=None):
-        if self.fused:
+        if self.mode == "streamed":
+            for L in self.layers:
+                self.layer_step_streamed(L, keep)
+        elif self.mode == "fused":
             tern.tern_act_stats(self.x, self.st_x)
             for L in self.layers:
                 self.layer_step_fused(L, keep)
@@ -156,7 +191,7 @@ class DecodeModel:
                 self.layer_step(L, keep)
 
     def capture(self) -> torch.cuda.CUDAGraph:
-        """One CUDA graph holding the whole step (8 launches per layer)."""
+        """One CUDA graph holding the whole step."""
         s = torch.cuda.Stream()
         s.wait_stream(torch.cuda.current_stream())
         with torch.cuda.stream(s):

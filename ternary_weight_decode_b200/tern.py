@@ -41,6 +41,7 @@ class tern_matrix(ctypes.Structure):
         ("row_stride", ctypes.c_int64),
         ("packed", ctypes.c_void_p),
         ("scales", ctypes.c_void_p),
+        ("scales_tiled", ctypes.c_void_p),
         ("flags", ctypes.c_int32),
         ("reserved", ctypes.c_int32),
     ]
@@ -68,6 +69,8 @@ def lib() -> ctypes.CDLL:
                 "tern_packed_size": (ctypes.c_int, [i32, i32, i32, i32, ctypes.POINTER(i64),
                                                     ctypes.POINTER(sz), ctypes.POINTER(sz)]),
                 "tern_canonical_row_bytes": (ctypes.c_int, [i32, i32, ctypes.POINTER(i64)]),
+                "tern_tiled_scales_bytes": (ctypes.c_int, [i32, i32, i32, ctypes.POINTER(sz)]),
+                "tern_retile_scales": (ctypes.c_int, [pm, p, p]),
                 "tern_pack": (ctypes.c_int, [i32, p, i32, i32, p, i64, p, p]),
                 "tern_unpack": (ctypes.c_int, [pm, p, p, p]),
                 "tern_import": (ctypes.c_int, [i32, p, i32, i32, p, i64, p, p]),
@@ -80,6 +83,10 @@ def lib() -> ctypes.CDLL:
                 "tern_act_stats": (ctypes.c_int, [p, i32, i32, i32, p, i32, p]),
                 "tern_debug_mma_i8": (ctypes.c_int, [i32, p, i32, p, i32, p, i32, i32, p]),
                 "tern_debug_select_engine": (ctypes.c_int, [i32]),
+                "tern_stream_workspace_bytes": (ctypes.c_int, [i32, i32, i32, i32, ctypes.POINTER(sz)]),
+                "tern_gemv_streamed": (ctypes.c_int, [pm, p, i32, i32, i32, p, p, i32, p, sz, p]),
+                "tern_gateup_swiglu_streamed": (ctypes.c_int, [pm, pm, p, i32, i32, i32, p, i32, p, sz,
+                                                               p]),
                 "tern_gemv_fused": (ctypes.c_int, [pm, p, i32, p, i32, i32, i32, p, p, i32, p, i32, p]),
                 "tern_gateup_swiglu_fused": (ctypes.c_int, [pm, pm, p, i32, p, i32, i32, i32, p, i32,
                                                             p, i32, p]),
@@ -127,6 +134,18 @@ def tern_canonical_row_bytes(fmt: int, K: int) -> int:
     return b.value
 
 
+def tern_tiled_scales_bytes(fmt: int, N: int, K: int) -> int:
+    b = ctypes.c_size_t()
+    _check(lib().tern_tiled_scales_bytes(fmt, N, K, ctypes.byref(b)), "tern_tiled_scales_bytes")
+    return b.value
+
+
+def tern_retile_scales(W, out: torch.Tensor, stream=None):
+    s = W.struct()
+    _check(lib().tern_retile_scales(ctypes.byref(s), _ptr(out), _stream(stream)),
+           "tern_retile_scales")
+
+
 # ------------------------------------------------------------------ matrices
 @dataclass
 class TernMatrix:
@@ -138,11 +157,20 @@ class TernMatrix:
     packed: torch.Tensor
     scales: torch.Tensor
     static: bool = True
+    scales_tiled: torch.Tensor | None = None
 
     def struct(self) -> tern_matrix:
         return tern_matrix(self.fmt, self.N, self.K, GROUP, self.row_stride,
                            self.packed.data_ptr(), self.scales.data_ptr(),
+                           None if self.scales_tiled is None else self.scales_tiled.data_ptr(),
                            TERN_MATRIX_STATIC if self.static else 0, 0)
+
+    def retile_scales(self, stream=None) -> "TernMatrix":
+        """Writes the unit-major copy of the scales the streamed kernels read."""
+        nbytes = tern_tiled_scales_bytes(self.fmt, self.N, self.K)
+        self.scales_tiled = torch.zeros(nbytes // 2, dtype=torch.float16, device=self.packed.device)
+        tern_retile_scales(self, self.scales_tiled, stream)
+        return self
 
     @staticmethod
     def empty(fmt: int, N: int, K: int, device="cuda") -> "TernMatrix":
@@ -279,6 +307,44 @@ def tern_debug_mma_i8(A: torch.Tensor, B: torch.Tensor, D: torch.Tensor, a_in_sm
     _check(lib().tern_debug_mma_i8(1 if a_in_smem else 0, _ptr(A), 1 if a_signed else 0, _ptr(B),
                                    1 if b_signed else 0, _ptr(D), K, N, _stream(stream)),
            "tern_debug_mma_i8")
+
+
+def tern_stream_workspace_bytes(fmt: int, N: int, M: int, two_matrices: bool) -> int:
+    b = ctypes.c_size_t()
+    _check(lib().tern_stream_workspace_bytes(fmt, N, M, 1 if two_matrices else 0, ctypes.byref(b)),
+           "tern_stream_workspace_bytes")
+    return b.value
+
+
+def stream_workspace(fmt: int, N: int, M: int, two_matrices: bool, device="cuda") -> torch.Tensor:
+    """A zeroed workspace for the streamed calls (kept zero by every call)."""
+    n = tern_stream_workspace_bytes(fmt, N, M, two_matrices)
+    return torch.zeros((n + 15) // 16 * 4, dtype=torch.int32, device=device)
+
+
+def tern_gemv_streamed(W: TernMatrix, x: torch.Tensor, y: torch.Tensor, workspace: torch.Tensor,
+                       qflags: int = 0, residual: torch.Tensor | None = None, M: int | None = None,
+                       stream=None):
+    M = x.shape[0] if M is None else M
+    assert x.dtype == torch.float32 and x.stride(1) == 1 and y.dtype == torch.float32
+    s = W.struct()
+    _check(lib().tern_gemv_streamed(ctypes.byref(s), _ptr(x), x.stride(0), qflags, M,
+                                    _ptr(residual), _ptr(y), y.stride(0), _ptr(workspace),
+                                    workspace.numel() * workspace.element_size(), _stream(stream)),
+           "tern_gemv_streamed")
+
+
+def tern_gateup_swiglu_streamed(Wg: TernMatrix, Wu: TernMatrix, x: torch.Tensor, h: torch.Tensor,
+                                workspace: torch.Tensor, qflags: int = 0, M: int | None = None,
+                                stream=None):
+    M = x.shape[0] if M is None else M
+    assert x.dtype == torch.float32 and x.stride(1) == 1 and h.dtype == torch.float32
+    sg, su = Wg.struct(), Wu.struct()
+    _check(lib().tern_gateup_swiglu_streamed(ctypes.byref(sg), ctypes.byref(su), _ptr(x),
+                                             x.stride(0), qflags, M, _ptr(h), h.stride(0),
+                                             _ptr(workspace),
+                                             workspace.numel() * workspace.element_size(),
+                                             _stream(stream)), "tern_gateup_swiglu_streamed")
 
 
 ENGINE_TENSOR_CORES, ENGINE_CUDA_CORES = 0, 1

@@ -42,8 +42,8 @@ def test_status_strings():
 
 def _matrix(**kw):
     from ternary_weight_decode_b200.tern import tern_matrix
-    base = dict(fmt=0, N=4, K=256, group=128, row_stride=64, packed=4096, scales=8192, flags=0,
-                reserved=0)
+    base = dict(fmt=0, N=4, K=256, group=128, row_stride=64, packed=4096, scales=8192,
+                scales_tiled=None, flags=0, reserved=0)
     base.update(kw)
     return tern_matrix(**base)
 

@@ -65,8 +65,9 @@ def check_layer(rec, l, rng, nrows=48):
 
 
 @pytest.mark.parametrize("fmt", [tern.TERN_FMT_BASE3, tern.TERN_FMT_2BIT])
-def test_decode_step_64_layers_sampled(fmt):
-    model = decode.DecodeModel(fmt, 64, M=1).build(seed_base=0)
+@pytest.mark.parametrize("mode", ["streamed", "fused"])
+def test_decode_step_64_layers_sampled(fmt, mode):
+    model = decode.DecodeModel(fmt, 64, M=1, mode=mode).build(seed_base=0)
     model.x.copy_(torch.from_numpy(synth.activations(0, 1, H).astype(np.float32)))
     rec = []
     model.step(keep=rec)
@@ -82,7 +83,8 @@ def test_decode_step_64_layers_sampled(fmt):
 
 @pytest.mark.parametrize("M", [2, 4, 16])
 def test_decode_layers_multi_slot(M):
-    model = decode.DecodeModel(tern.TERN_FMT_BASE3, 2, M=M).build(seed_base=0)
+    mode = "streamed" if M <= 2 else "fused"
+    model = decode.DecodeModel(tern.TERN_FMT_BASE3, 2, M=M, mode=mode).build(seed_base=0)
     x0 = synth.activation_rows([1000 + r for r in range(M)], H).astype(np.float32)
     model.x.copy_(torch.from_numpy(x0))
     rec = []
@@ -94,8 +96,9 @@ def test_decode_layers_multi_slot(M):
         check_layer(rec, l, rng, nrows=24)
 
 
-def test_graph_replay_matches_eager():
-    model = decode.DecodeModel(tern.TERN_FMT_BASE3, 3, M=1).build(seed_base=0)
+@pytest.mark.parametrize("mode", ["streamed", "fused"])
+def test_graph_replay_matches_eager(mode):
+    model = decode.DecodeModel(tern.TERN_FMT_BASE3, 3, M=1, mode=mode).build(seed_base=0)
     x0 = torch.from_numpy(synth.activations(3, 1, H).astype(np.float32)).cuda()
     model.x.copy_(x0)
     model.step()
