@@ -286,6 +286,32 @@ tern_status tern_gateup_swiglu_streamed(const tern_matrix *Wg, const tern_matrix
                                         void *stream);
 
 /*
+ * tern_gemv_streamed without a caller workspace (the pages have no
+ * counterpart: this is a convenience of the library).  Some callers cannot
+ * call cudaMalloc: a plug-in whose host program owns all device memory
+ * through its own pool or a fixed budget, or code on a latency-critical
+ * path where cudaMalloc's implicit device-wide synchronisation would stall
+ * other streams.  This entry point allocates nothing.  The kernel's scratch
+ * -- fp32 partial sums and arrival counters of the row blocks that two CTAs
+ * share -- is a fixed array of TERN_NOALLOC_SCRATCH_BYTES (1 MiB) inside the
+ * library, held on every GPU that loads the library until the process exits.
+ * Arguments, results and errors are those of tern_gemv_streamed.  Also:
+ *  - sizes whose scratch exceeds the array are rejected with TERN_EINVAL
+ *    (N <= 129024 at M = 1, N <= 65024 at M = 2);
+ *  - the first call on a device looks up the array's device address there
+ *    (that device current) and keeps it; make that first call before any
+ *    stream capture;
+ *  - each call clears the counters it uses (an asynchronous memset on
+ *    `stream`, then the kernel); every call on a device shares the one
+ *    array, so calls that may overlap on the GPU (other streams, other host
+ *    threads) race and give wrong results: serialise them.
+ */
+#define TERN_NOALLOC_SCRATCH_BYTES (1u << 20)
+tern_status tern_gemv_streamed_noalloc(const tern_matrix *W, const float *x, int32_t ldx,
+                                       int32_t qflags, int32_t M, const float *residual,
+                                       float *y, int32_t ldy, void *stream);
+
+/*
  * Test hook for the tensor-core path (no counterpart on the pages; it pins
  * the tcgen05 encodings the kernels use): one CTA computes
  *   D[m][n] = sum_k A[m][k] * B[n][k]   (int32, exact)

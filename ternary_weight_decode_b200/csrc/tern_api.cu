@@ -56,6 +56,13 @@ tern_status check_activations(const int8_t *q, int32_t ldq, int32_t K, const flo
 
 }  // namespace
 
+namespace tern {
+tern_status set_last_error(tern_status s, const char *message) {
+    snprintf(g_last_error, sizeof(g_last_error), "%s", message);
+    return s;
+}
+}  // namespace tern
+
 extern "C" {
 
 const char *tern_status_string(tern_status s) {

@@ -103,6 +103,9 @@ cudaError_t launch_act_stats(const float *x, int M, int K, int ldx, float *stats
                              cudaStream_t s);
 cudaError_t read_clear_device_error(int *value, cudaStream_t s);
 
+// Sets the message tern_last_error() returns on the calling host thread.
+tern_status set_last_error(tern_status s, const char *message);
+
 // ---------------------------------------------------------------- tcgen05 test hook
 cudaError_t launch_debug_mma(int a_in_smem, const int8_t *A, int a_signed, const int8_t *B,
                              int b_signed, int32_t *D, int K, int N, cudaStream_t s);

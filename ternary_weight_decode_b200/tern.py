@@ -87,6 +87,7 @@ def lib() -> ctypes.CDLL:
                 "tern_gemv_streamed": (ctypes.c_int, [pm, p, i32, i32, i32, p, p, i32, p, sz, p]),
                 "tern_gateup_swiglu_streamed": (ctypes.c_int, [pm, pm, p, i32, i32, i32, p, i32, p, sz,
                                                                p]),
+                "tern_gemv_streamed_noalloc": (ctypes.c_int, [pm, p, i32, i32, i32, p, p, i32, p]),
                 "tern_gemv_fused": (ctypes.c_int, [pm, p, i32, p, i32, i32, i32, p, p, i32, p, i32, p]),
                 "tern_gateup_swiglu_fused": (ctypes.c_int, [pm, pm, p, i32, p, i32, i32, i32, p, i32,
                                                             p, i32, p]),
@@ -332,6 +333,23 @@ def tern_gemv_streamed(W: TernMatrix, x: torch.Tensor, y: torch.Tensor, workspac
                                     _ptr(residual), _ptr(y), y.stride(0), _ptr(workspace),
                                     workspace.numel() * workspace.element_size(), _stream(stream)),
            "tern_gemv_streamed")
+
+
+# Size of the scratch array tern_gemv_streamed_noalloc uses (include/tern.h).
+NOALLOC_SCRATCH_BYTES = 1 << 20
+
+
+def tern_gemv_streamed_noalloc(W: TernMatrix, x: torch.Tensor, y: torch.Tensor, qflags: int = 0,
+                               residual: torch.Tensor | None = None, M: int | None = None,
+                               stream=None):
+    """tern_gemv_streamed with the library's own scratch array in place of a
+    caller workspace: for callers that cannot allocate device memory."""
+    M = x.shape[0] if M is None else M
+    assert x.dtype == torch.float32 and x.stride(1) == 1 and y.dtype == torch.float32
+    s = W.struct()
+    _check(lib().tern_gemv_streamed_noalloc(ctypes.byref(s), _ptr(x), x.stride(0), qflags, M,
+                                            _ptr(residual), _ptr(y), y.stride(0), _stream(stream)),
+           "tern_gemv_streamed_noalloc")
 
 
 def tern_gateup_swiglu_streamed(Wg: TernMatrix, Wu: TernMatrix, x: torch.Tensor, h: torch.Tensor,
