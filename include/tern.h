@@ -196,6 +196,25 @@ tern_status tern_gemv(const tern_matrix *W, const int8_t *q, int32_t ldq,
                       float *y, int32_t ldy, void *stream);
 
 /*
+ * Prefill GEMM on the tensor cores (Bonsai page, "Decode 为什么只能算一般":
+ * prefill is a large matrix multiply over the same packed weights), any
+ * number of token rows M >= 1:
+ *   y[m][n] = s_x[m] * sum_g s_w[n][g] * P[m][n][g],
+ *   P[m][n][g] = sum_{k in group g} w[n][k] * q[m][k]   (exact int32),
+ * the product of tern_gemv without a residual.  The trits are expanded to
+ * int8 in shared memory and multiplied by tcgen05.mma kind::i8 into int32
+ * tensor memory, one 128-K group at a time; the fp32 epilogue applies the
+ * group scales in group order.
+ *  q: device int8 [M][ldq], 16-byte aligned, ldq >= K, ldq % 16 == 0
+ *     (bytes past K are ignored).  s_x: device fp32 [M].
+ *  y: device fp32 [M][ldy], ldy >= N; must not overlap q.
+ * The caller owns every buffer; nothing is allocated.
+ */
+tern_status tern_gemm(const tern_matrix *W, const int8_t *q, int32_t ldq,
+                      const float *s_x, int32_t M, float *y, int32_t ldy,
+                      void *stream);
+
+/*
  * Fused gate/up + SwiGLU (Bonsai page, "Decode 为什么只能算一般"):
  *   g = Wg x^, u = Wu x^ (each as in tern_gemv, same q and s_x),
  *   h[m][n] = g * sigmoid(g) * u,  sigmoid(z) = 1/(1+exp(-z)).
@@ -262,13 +281,13 @@ tern_status tern_gateup_swiglu_fused(const tern_matrix *Wg, const tern_matrix *W
  *    scale from x itself (max |x|, or max |H x| with TERN_QUANT_FWHT128);
  *  - W->scales_tiled must hold the re-tiled scales (tern_retile_scales);
  *  - workspace: device, 16-byte aligned, >= tern_stream_workspace_bytes()
- *    bytes, all zero before its first use.  It holds fp32 partial sums
- *    (scratch) from its start and one int32 arrival counter per 32-row
- *    block from its end backwards (block rb at byte ws_bytes - 4 (rb + 1),
- *    ws_bytes rounded down to a multiple of 4); every call leaves the
- *    counters zero again, so one workspace, sized for the largest call,
- *    serves a whole chain of calls of any sizes on one stream (calls that
- *    may overlap need separate workspaces).
+ *    bytes, all zero before its first use.  It carries, from its start, the
+ *    partial sums of the 32-row blocks that two CTAs share (one 64-bit word
+ *    per row, matrix and token: fp32 value and a tag); every call clears
+ *    what it wrote, so the workspace is all zero again after each call and
+ *    one workspace, sized for the largest call, serves a whole chain of
+ *    calls of any sizes on one stream (calls that may overlap need separate
+ *    workspaces).
  * One CTA per SM streams an equal share of the matrix's 32-row x 128-byte
  * tiles; with TERN_MATRIX_STATIC the tiles start streaming before the
  * previous kernel on the stream has finished.  x must not overlap y / h.
@@ -292,8 +311,7 @@ tern_status tern_gateup_swiglu_streamed(const tern_matrix *Wg, const tern_matrix
  * through its own pool or a fixed budget, or code on a latency-critical
  * path where cudaMalloc's implicit device-wide synchronisation would stall
  * other streams.  This entry point allocates nothing.  The kernel's scratch
- * -- fp32 partial sums and arrival counters of the row blocks that two CTAs
- * share -- is a fixed array of TERN_NOALLOC_SCRATCH_BYTES (1 MiB) inside the
+ * -- the partial sums of the row blocks that two CTAs share -- is a fixed array of TERN_NOALLOC_SCRATCH_BYTES (1 MiB) inside the
  * library, held on every GPU that loads the library until the process exits.
  * Arguments, results and errors are those of tern_gemv_streamed.  Also:
  *  - sizes whose scratch exceeds the array are rejected with TERN_EINVAL
@@ -301,10 +319,10 @@ tern_status tern_gateup_swiglu_streamed(const tern_matrix *Wg, const tern_matrix
  *  - the first call on a device looks up the array's device address there
  *    (that device current) and keeps it; make that first call before any
  *    stream capture;
- *  - each call clears the counters it uses (an asynchronous memset on
- *    `stream`, then the kernel); every call on a device shares the one
- *    array, so calls that may overlap on the GPU (other streams, other host
- *    threads) race and give wrong results: serialise them.
+ *  - each call first clears the part of the array it uses (an asynchronous
+ *    memset on `stream`, then the kernel); every call on a device shares
+ *    the one array, so calls that may overlap on the GPU (other streams,
+ *    other host threads) race and give wrong results: serialise them.
  */
 #define TERN_NOALLOC_SCRATCH_BYTES (1u << 20)
 tern_status tern_gemv_streamed_noalloc(const tern_matrix *W, const float *x, int32_t ldx,
@@ -317,7 +335,9 @@ tern_status tern_gemv_streamed_noalloc(const tern_matrix *W, const float *x, int
  *   D[m][n] = sum_k A[m][k] * B[n][k]   (int32, exact)
  * for A int8 [128][K] (row-major; read as unsigned bytes when a_signed == 0)
  * and B int8 [N][K] (row-major; unsigned when b_signed == 0), with A taken
- * from tensor memory (a_in_smem == 0) or shared memory (1).
+ * from tensor memory (a_in_smem == 0) or shared memory (1), B from shared
+ * memory without swizzle; mode 2: A and B both from shared memory in the
+ * 128-byte-swizzled K-major layout of tern_gemm (then K % 128 == 0).
  * K in 32..512, a multiple of 32; N in 16..256, a multiple of 16.
  * A, B: device, 16-byte aligned; D: device int32 [128][N].
  */

@@ -307,7 +307,10 @@ tern_status tern_debug_mma_i8(int32_t a_in_smem, const int8_t *A, int32_t a_sign
     if (N < 16 || N > 256 || N % 16 != 0) return fail(TERN_EINVAL, "tern_debug_mma_i8: N must be 16..256, a multiple of 16%s");
     if (!A || !B || !D || !aligned(A, 16) || !aligned(B, 16) || !aligned(D, 16))
         return fail(TERN_EINVAL, "tern_debug_mma_i8: pointers must be 16-byte aligned%s");
-    return cuda_status(tern::launch_debug_mma(a_in_smem ? 1 : 0, A, a_signed ? 1 : 0, B, b_signed ? 1 : 0,
+    if (a_in_smem < 0 || a_in_smem > 2) return fail(TERN_EINVAL, "tern_debug_mma_i8: mode must be 0, 1 or 2%s");
+    if (a_in_smem == 2 && K % 128 != 0)
+        return fail(TERN_EINVAL, "tern_debug_mma_i8: mode 2 needs K %% 128 == 0%s");
+    return cuda_status(tern::launch_debug_mma(a_in_smem, A, a_signed ? 1 : 0, B, b_signed ? 1 : 0,
                                               D, K, N, static_cast<cudaStream_t>(stream)),
                        "tern_debug_mma_i8");
 }
@@ -391,6 +394,35 @@ tern_status tern_gateup_swiglu_streamed(const tern_matrix *Wg, const tern_matrix
         return fail(TERN_EINVAL, "tern_gateup_swiglu_streamed: gate and up must share fmt, N, K, group, row_stride%s");
     return run_streamed(Wg, Wu, x, ldx, qflags, M, nullptr, h, ldh, workspace, ws_bytes, stream,
                         "tern_gateup_swiglu_streamed");
+}
+
+tern_status tern_gemm(const tern_matrix *W, const int8_t *q, int32_t ldq, const float *s_x,
+                      int32_t M, float *y, int32_t ldy, void *stream) {
+    tern_status st = check_matrix(W, "tern_gemm");
+    if (st != TERN_OK) return st;
+    if (M < 1) return fail(TERN_EINVAL, "tern_gemm: M must be >= 1%s");
+    if (!q || !aligned(q, 16) || ldq < W->K || ldq % 16 != 0)
+        return fail(TERN_EINVAL, "tern_gemm: q must be 16-byte aligned with ldq >= K, ldq %% 16 == 0%s");
+    if (!s_x || !aligned(s_x, 4)) return fail(TERN_EINVAL, "tern_gemm: bad s_x%s");
+    if (!y || !aligned(y, 4) || ldy < W->N) return fail(TERN_EINVAL, "tern_gemm: bad y or ldy%s");
+    tern::GemmLaunch L = {};
+    L.fmt = W->fmt;
+    L.N = W->N;
+    L.K = W->K;
+    L.M = M;
+    L.row_bytes = tern::device_row_bytes(W->fmt, W->K);
+    L.row_stride = W->row_stride;
+    L.packed = W->packed;
+    L.scales = W->scales;
+    L.q = q;
+    L.ldq = ldq;
+    L.s_x = s_x;
+    L.y = y;
+    L.ldy = ldy;
+    const char *why = nullptr;
+    cudaError_t e = tern::launch_gemm(L, static_cast<cudaStream_t>(stream), &why);
+    if (why) return fail(TERN_EUNSUPPORTED, "tern_gemm: %s", why);
+    return cuda_status(e, "tern_gemm");
 }
 
 tern_status tern_debug_select_engine(int32_t engine) {

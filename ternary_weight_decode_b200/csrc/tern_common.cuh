@@ -42,6 +42,10 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t *bar, uint32_t by
                  : "memory");
 }
 
+__device__ __forceinline__ void mbar_arrive(uint64_t *bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
 __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
     uint32_t ok;
     asm volatile(
@@ -88,6 +92,16 @@ __device__ __forceinline__ void tma_load_2d(void *smem_dst, const CUtensorMap *m
         : "memory");
 }
 
+// The same without a cache hint (operands that other CTAs read again).
+__device__ __forceinline__ void tma_load_2d_nohint(void *smem_dst, const CUtensorMap *map, int x, int y,
+                                                   uint64_t *bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%2, %3}], [%4];" ::"r"(smem_u32(smem_dst)),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_u32(bar))
+        : "memory");
+}
+
 // L2 policy for data read exactly once (the weight stream).
 __device__ __forceinline__ uint64_t l2_policy_evict_first() {
     uint64_t p;
@@ -114,6 +128,88 @@ __device__ __forceinline__ uint32_t map_shared_rank(const void *p, uint32_t rank
     uint32_t out;
     asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(out) : "r"(smem_u32(p)), "r"(rank));
     return out;
+}
+
+__device__ __forceinline__ uint32_t cluster_nctarank() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_nctarank;" : "=r"(r));
+    return r;
+}
+
+// Split cluster barrier: every thread of every CTA of the cluster arrives
+// once, and may wait later.
+__device__ __forceinline__ void cluster_arrive() {
+    asm volatile("barrier.cluster.arrive.release;" ::: "memory");
+}
+__device__ __forceinline__ void cluster_wait() {
+    asm volatile("barrier.cluster.wait.acquire;" ::: "memory");
+}
+
+// Asynchronous store of 4 / 8 bytes into the shared memory of a CTA of the
+// cluster (addresses from map_shared_rank); completes the bytes on that
+// CTA's mbarrier `remote_bar`.
+__device__ __forceinline__ void st_async_u32(uint32_t remote_addr, uint32_t v, uint32_t remote_bar) {
+    asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.u32 [%0], %1, [%2];" ::"r"(
+                     remote_addr),
+                 "r"(v), "r"(remote_bar)
+                 : "memory");
+}
+__device__ __forceinline__ void st_async_v2f32(uint32_t remote_addr, float a, float b,
+                                               uint32_t remote_bar) {
+    asm volatile(
+        "st.async.shared::cluster.mbarrier::complete_tx::bytes.v2.f32 [%0], {%1, %2}, [%3];" ::"r"(
+            remote_addr),
+        "f"(a), "f"(b), "r"(remote_bar)
+        : "memory");
+}
+
+// Bulk copy of `bytes` (multiple of 16, both addresses 16-byte aligned) from
+// this CTA's shared memory into the shared memory of a CTA of the cluster,
+// completing the bytes on that CTA's mbarrier.  The source must have been
+// made visible to the async proxy (fence_proxy_async_smem) by its writers.
+__device__ __forceinline__ void bulk_copy_s2cluster(uint32_t remote_dst, const void *src,
+                                                    uint32_t bytes, uint32_t remote_bar) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.shared::cta.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+            remote_dst),
+        "r"(smem_u32(src)), "r"(bytes), "r"(remote_bar)
+        : "memory");
+}
+
+// 8-byte relaxed accesses at GPU scope: single-copy atomic, so a (value,
+// tag) pair packed into one 64-bit word is seen whole or not at all.
+__device__ __forceinline__ void st_relaxed_gpu_u64(unsigned long long *p, unsigned long long v) {
+    asm volatile("st.relaxed.gpu.global.b64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
+}
+__device__ __forceinline__ unsigned long long ld_relaxed_gpu_u64(const unsigned long long *p) {
+    unsigned long long v;
+    asm volatile("ld.relaxed.gpu.global.b64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
+    return v;
+}
+
+// Waits (bounded, like mbar_wait_bounded) for a phase completed by other CTAs
+// of the cluster, with acquire at cluster scope.
+__device__ __forceinline__ bool mbar_try_wait_cluster(uint64_t *bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+__device__ __forceinline__ bool mbar_wait_cluster_bounded(uint64_t *bar, uint32_t parity) {
+    if (mbar_try_wait_cluster(bar, parity)) return true;
+    long long start = clock64();
+    while (!mbar_try_wait_cluster(bar, parity)) {
+        if (clock64() - start > kWaitBudgetCycles) {
+            atomicExch(&g_device_error, kErrTmaTimeout);
+            return false;
+        }
+    }
+    return true;
 }
 
 __device__ __forceinline__ float ld_shared_cluster_f32(uint32_t addr) {

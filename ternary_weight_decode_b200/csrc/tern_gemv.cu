@@ -457,18 +457,24 @@ int g_engine = 1;  // 0: tensor cores, 1: CUDA cores (default); set by a test ho
 
 }  // namespace
 
-bool make_weight_tmap(CUtensorMap *map, const void *packed, int64_t row_bytes, int N,
-                      int64_t row_stride) {
+bool make_u8_tmap_2d(CUtensorMap *map, const void *base, uint64_t inner, uint64_t rows,
+                     uint64_t stride, uint32_t box_inner, uint32_t box_rows) {
     EncodeTiledFn fn = encode_fn();
     if (!fn) return false;
-    cuuint64_t dims[2] = {static_cast<cuuint64_t>(row_bytes), static_cast<cuuint64_t>(N)};
-    cuuint64_t strides[1] = {static_cast<cuuint64_t>(row_stride)};
-    cuuint32_t box[2] = {kSBBytes, 32};
+    cuuint64_t dims[2] = {static_cast<cuuint64_t>(inner), static_cast<cuuint64_t>(rows)};
+    cuuint64_t strides[1] = {static_cast<cuuint64_t>(stride)};
+    cuuint32_t box[2] = {box_inner, box_rows};
     cuuint32_t estr[2] = {1, 1};
-    CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void *>(packed), dims, strides,
+    CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void *>(base), dims, strides,
                     box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS;
+}
+
+bool make_weight_tmap(CUtensorMap *map, const void *packed, int64_t row_bytes, int N,
+                      int64_t row_stride) {
+    return make_u8_tmap_2d(map, packed, static_cast<uint64_t>(row_bytes), static_cast<uint64_t>(N),
+                           static_cast<uint64_t>(row_stride), kSBBytes, 32);
 }
 
 void fill_params(GemvParams &p, const GemvLaunch &L) {

@@ -6,29 +6,36 @@
 // FP16 group scale -- 4sapi page, section 三); this file changes how the
 // work is laid over the GPU so that one projection costs about its bytes:
 //
-//  * A "unit" is 32 rows x one 128-byte superblock of codes.  The U units of
-//    a matrix (row-block major) are cut into equal contiguous ranges, one per
-//    CTA, one CTA per SM -- so every SM streams the same number of bytes.
+//  * A "unit" is 32 rows x one 128-byte superblock of codes; an "item" is one
+//    unit of one matrix (gate and up are two items of the same unit).  The
+//    units of a matrix (row-block major) are cut into equal contiguous ranges,
+//    one per CTA, one CTA per SM -- so every SM streams the same bytes.
 //  * Warp 0 of a CTA is a producer: from the first instruction (before the
 //    previous kernel on the stream has finished, when the matrix is static)
-//    it streams its units into a ring of shared-memory slots: the 32 x 128 B
-//    code tile by TMA (128-byte swizzle, L2 evict-first, no multicast) and
-//    the unit's 32 x GPS scales, re-tiled at load time into unit order, by a
-//    bulk copy.  A CTA of the next kernel, resident beside this one under
+//    it streams its items into a ring of shared-memory slots: the 32 x 128 B
+//    code tile by TMA (128-byte swizzle, L2 evict-first, no multicast) and the
+//    unit's 32 x GPS scales, re-tiled at load time into unit order, by a bulk
+//    copy.  A CTA of the next kernel, resident beside this one under
 //    programmatic dependent launch, fills its own ring meanwhile.
-//  * Warps 1..8 are consumers.  After the previous kernel finishes they
-//    quantise the fp32 input once per CTA (two passes: row scale from max|x|
-//    -- or max|H x| with the Hadamard rotation -- then the int8 codes and
-//    per-group sums), then take units round-robin: lane = row, decode +
-//    dp4a as in tern_gemv.cu, one fp32 partial per (unit, row).
+//  * Warps 1..8 are consumers.  The input is quantised once per cluster of C
+//    CTAs: each CTA takes 1/C of the 128-blocks of the fp32 input, forms its
+//    share of max |x| (max |H x| with the Hadamard rotation) and of sum x^2,
+//    sends it to every CTA of the cluster (st.async into their shared
+//    memory), then quantises its blocks with the cluster-wide row scale and
+//    sends the int8 codes and group sums to every CTA the same way.
+//  * Consumers then take items round-robin: lane = row; the item's codes and
+//    scales are copied to registers and the ring slot is handed back at once,
+//    so the whole ring stays in flight; decode + dp4a as in tern_gemv.cu; one
+//    fp32 partial per (item, row, token).
 //  * Row blocks inside a CTA's range are summed in unit order and written.
-//    A row block cut by a range boundary belongs to two CTAs: each writes
-//    its partial to the workspace (from its start) and increments the row
-//    block's counter (counters sit at the end of the workspace, so calls of
-//    any size that share it agree on where each counter is);
-//    the second one adds lower + upper (fixed order, so the result does not
-//    depend on which finishes first), writes the output and resets the
-//    counter, so the workspace is zero again for the next call.
+//    A row block cut by a range boundary belongs to two CTAs.  The one that
+//    holds its end (its first units) publishes its partial as soon as those
+//    units are done: value and tag in one 64-bit store into the workspace.
+//    The one that holds its start adds that partial to its own at its end
+//    (lower + upper: fixed order, so the result does not depend on timing)
+//    with one relaxed 64-bit load, waiting (bounded) only if the tag is not
+//    there yet, then clears the word -- the workspace is zero again after
+//    every call.
 #include "tern_gemv_common.cuh"
 
 namespace tern {
@@ -36,19 +43,19 @@ namespace {
 
 constexpr int kSkConsumers = 8;
 constexpr int kSkThreads = 32 * (kSkConsumers + 1);
-constexpr int kSkBar = 1;  // named barrier of the consumer warps
+constexpr int kSkBar = 1;   // named barrier of the consumer warps
+constexpr int kSkKeep = 5;  // input blocks a consumer warp keeps in registers
+constexpr int kSkMaxCluster = 4;
+constexpr int kSkSmemBudget = 112 * 1024;  // two CTAs per SM (programmatic launch overlap)
+constexpr int kSkMinRing = 8, kSkMaxRing = 24;
 
 template <int FMT>
 __host__ __device__ constexpr int scb() {
     return 32 * Fmt<FMT>::kGroups * 2;  // bytes of one unit's scales
 }
-template <int NMAT>
-__host__ __device__ constexpr int sk_ring() {
-    return NMAT == 1 ? 16 : 8;
-}
 
 struct SkParams {
-    int N, K, G, SB, RB;
+    int N, K, SB, RB, R;
     long long U;
     int nCTA, M, prefetch_ok, qflags;
     const uint16_t *tsc0;
@@ -58,37 +65,43 @@ struct SkParams {
     const float *residual;
     float *out;
     int ldo;
-    float *ws_part;
-    int *ws_cnt_end;  // counter of row block rb is ws_cnt_end[-1 - rb]
+    unsigned long long *ws_tag;  // tagged partials of cut row blocks, zero at rest
 };
 
 struct SkLayout {
-    int ring_s_off, act_off, sq_off, sx_off, red_off, slots_off, bar_off, total;
-    int Kpad, GT, umax;
+    int ring_s_off, act_off, sq_off, xred_off, sx_off, red_off, misc_off, slots_off, bar_off, total;
+    int Kpad, GT;
 };
 
-template <int FMT, int MT, int NMAT>
-__host__ __device__ inline SkLayout sk_layout(int SB, int umax) {
-    constexpr int R = sk_ring<NMAT>();
+// Shared memory plan: ring of R slots (code tile + scales), the int8 input
+// over the padded K (MT rows), its group sums (one per 16 bytes, so that a
+// CTA's share is one aligned bulk copy), the cluster's partials of the row
+// scale, row scales, per-warp partials, a counter, per-(item, token) row
+// partials, barriers.
+template <int FMT, int MT>
+__host__ __device__ inline SkLayout sk_layout(int SB, int items_max, int R) {
     SkLayout L;
     L.Kpad = SB * Fmt<FMT>::kPos;
-    L.GT = SB * Fmt<FMT>::kGroups;
-    L.umax = umax;
-    int off = R * NMAT * kTile;  // code tiles, 1024-aligned slots (128-byte swizzle)
+    L.GT = SB * Fmt<FMT>::kGroups;  // 128-blocks of the padded K
+    int off = R * kTile;            // code tiles, 1024-aligned slots (128-byte swizzle)
     L.ring_s_off = off;
-    off = align128(off + R * NMAT * scb<FMT>());
+    off = align128(off + R * scb<FMT>());
     L.act_off = off;
     off = align128(off + MT * L.Kpad);
     L.sq_off = off;
-    off = align128(off + MT * L.GT * 4);
+    off = align128(off + MT * L.GT * 16);
+    L.xred_off = off;
+    off = align128(off + kSkMaxCluster * MT * 2 * 4);
     L.sx_off = off;
     off = align128(off + 2 * MT * 4);
     L.red_off = off;
     off = align128(off + kSkConsumers * MT * 2 * 4);
+    L.misc_off = off;
+    off = align128(off + 16);
     L.slots_off = off;
-    off = align128(off + umax * NMAT * MT * 32 * 4);
+    off = align128(off + items_max * MT * 32 * 4);
     L.bar_off = off;
-    off += 2 * R * 8;
+    off += (2 * R + 2) * 8;
     L.total = off + 1024;
     return L;
 }
@@ -102,63 +115,35 @@ __device__ __forceinline__ void bulk_copy_g2s(void *dst, const void *src, uint32
         : "memory");
 }
 
-__device__ __forceinline__ void mbar_arrive(uint64_t *bar) {
-    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
-}
-
-__device__ __forceinline__ float unit_scale(const uint8_t *s, int lane, int gps, int g) {
-    return __half2float(
-        __ushort_as_half(reinterpret_cast<const uint16_t *>(s)[lane * gps + g]));
-}
-
-// One unit (this lane's row, one superblock) of NMAT matrices: the decode and
-// dp4a of tern_gemv.cu with the unit's scales from its ring slot.
-template <int FMT, int MT, int NMAT>
-__device__ __forceinline__ void sk_unit(const uint8_t *wtile, const uint8_t *stile, int lane,
-                                        const uint8_t *act_sb, int Kpad, const int *sq_sb, int GT,
-                                        float (&yacc)[NMAT][MT]) {
-    constexpr int GPS = Fmt<FMT>::kGroups;
-    constexpr int SCB = scb<FMT>();
-    const int rsw = lane & 7;
-    int acc[NMAT][MT];
+// One item (this lane's row, one superblock of one matrix) from registers:
+// the decode and dp4a of tern_gemv.cu.  words: the row's 128 code bytes in
+// K order; sc: the row's GPS group scales; sq_sb: group sums of the input,
+// one per 4 ints.
+template <int FMT, int MT>
+__device__ __forceinline__ void sk_item(const uint32_t (&words)[32],
+                                        const float (&sc)[Fmt<FMT>::kGroups], const uint8_t *act_sb,
+                                        int Kpad, const int *sq_sb, int GT, float (&yacc)[MT]) {
+    int acc[MT];
 #pragma unroll
-    for (int mat = 0; mat < NMAT; ++mat)
-#pragma unroll
-        for (int m = 0; m < MT; ++m) {
-            acc[mat][m] = 0;
-            yacc[mat][m] = 0.0f;
-        }
+    for (int m = 0; m < MT; ++m) {
+        acc[m] = 0;
+        yacc[m] = 0.0f;
+    }
     auto finish = [&](int m, int g) {
-        const int s = sq_sb[m * GT + g];
-#pragma unroll
-        for (int mat = 0; mat < NMAT; ++mat) {
-            yacc[mat][m] = fmaf(unit_scale(stile + mat * SCB, lane, GPS, g),
-                                static_cast<float>(acc[mat][m] - s), yacc[mat][m]);
-            acc[mat][m] = 0;
-        }
+        yacc[m] = fmaf(sc[g], static_cast<float>(acc[m] - sq_sb[(m * GT + g) * 4]), yacc[m]);
+        acc[m] = 0;
     };
 #pragma unroll
     for (int c = 0; c < 8; ++c) {
-        uint32_t words[NMAT][4];
-#pragma unroll
-        for (int mat = 0; mat < NMAT; ++mat) {
-            const uint4 wv = lds128(wtile + mat * kTile + lane * kSBBytes + ((c ^ rsw) << 4));
-            words[mat][0] = wv.x;
-            words[mat][1] = wv.y;
-            words[mat][2] = wv.z;
-            words[mat][3] = wv.w;
-        }
         if constexpr (FMT == TERN_FMT_BASE3) {
-            uint32_t t[NMAT][20];
+            uint32_t t[20];
 #pragma unroll
-            for (int mat = 0; mat < NMAT; ++mat)
+            for (int wi = 0; wi < 4; ++wi) {
+                uint32_t tw[5];
+                decode_d3(words[4 * c + wi], tw);
 #pragma unroll
-                for (int wi = 0; wi < 4; ++wi) {
-                    uint32_t tw[5];
-                    decode_d3(words[mat][wi], tw);
-#pragma unroll
-                    for (int i = 0; i < 5; ++i) t[mat][5 * wi + i] = tw[i];
-                }
+                for (int i = 0; i < 5; ++i) t[5 * wi + i] = tw[i];
+            }
 #pragma unroll
             for (int m = 0; m < MT; ++m) {
                 const uint8_t *a = act_sb + m * Kpad + c * 80;
@@ -175,8 +160,7 @@ __device__ __forceinline__ void sk_unit(const uint8_t *wtile, const uint8_t *sti
                 for (int d = 0; d < 20; ++d) {
                     const int dd = c * 20 + d;
                     if (dd > 0 && (dd & 31) == 0) finish(m, (dd >> 5) - 1);
-#pragma unroll
-                    for (int mat = 0; mat < NMAT; ++mat) acc[mat][m] = dp4a_ss(t[mat][d], aw[d], acc[mat][m]);
+                    acc[m] = dp4a_ss(t[d], aw[d], acc[m]);
                 }
             }
         } else {
@@ -192,16 +176,14 @@ __device__ __forceinline__ void sk_unit(const uint8_t *wtile, const uint8_t *sti
                     aw[4 * j + 2] = v.z;
                     aw[4 * j + 3] = v.w;
                 }
+                int a4[4] = {0, 0, 0, 0};
 #pragma unroll
-                for (int mat = 0; mat < NMAT; ++mat) {
-                    int a4[4] = {0, 0, 0, 0};
+                for (int wi = 0; wi < 4; ++wi)
 #pragma unroll
-                    for (int wi = 0; wi < 4; ++wi)
-#pragma unroll
-                        for (int i = 0; i < 4; ++i)
-                            a4[i] = dp4a_us(words[mat][wi] & (0x03030303u << (2 * i)), aw[4 * wi + i], a4[i]);
-                    acc[mat][m] += a4[0] + (a4[1] >> 2) + (a4[2] >> 4) + (a4[3] >> 6);
-                }
+                    for (int i = 0; i < 4; ++i)
+                        a4[i] = dp4a_us(words[4 * c + wi] & (0x03030303u << (2 * i)), aw[4 * wi + i],
+                                        a4[i]);
+                acc[m] += a4[0] + (a4[1] >> 2) + (a4[2] >> 4) + (a4[3] >> 6);
                 if (c & 1) finish(m, c >> 1);
             }
         }
@@ -212,34 +194,73 @@ __device__ __forceinline__ void sk_unit(const uint8_t *wtile, const uint8_t *sti
     }
 }
 
+// Lane's 4 values of 128-block b of token row m (zero past K and for m >= M).
+__device__ __forceinline__ void load_block(const SkParams &p, int m, int b, int lane, float (&r)[4]) {
+    r[0] = r[1] = r[2] = r[3] = 0.0f;
+    const int k = 128 * b + 4 * lane;
+    if (m >= p.M || k >= p.K) return;
+    const float *src = p.x + static_cast<int64_t>(m) * p.ldx + k;
+    if (k + 4 <= p.K) {
+        const float4 v = __ldcg(reinterpret_cast<const float4 *>(src));
+        r[0] = v.x;
+        r[1] = v.y;
+        r[2] = v.z;
+        r[3] = v.w;
+    } else {
+        for (int e = 0; e < 4 && k + e < p.K; ++e) r[e] = __ldcg(src + e);
+    }
+}
+
+__device__ __forceinline__ float sumsq4(const float (&r)[4]) {
+    return fmaf(r[3], r[3], fmaf(r[2], r[2], fmaf(r[1], r[1], r[0] * r[0])));
+}
+__device__ __forceinline__ float amax4(const float (&r)[4]) {
+    return fmaxf(fmaxf(fabsf(r[0]), fabsf(r[1])), fmaxf(fabsf(r[2]), fabsf(r[3])));
+}
+
+// Index of the tagged partial of (row block, matrix, token, lane).
+template <int NMAT, int MT>
+__device__ __forceinline__ int64_t tag_index(int rb, int mat, int m, int lane) {
+    return ((static_cast<int64_t>(rb) * NMAT + mat) * MT + m) * 32 + lane;
+}
+
 template <int FMT, int MT, int MODE>
-__global__ void __launch_bounds__(kSkThreads, 1)
+__global__ void __launch_bounds__(kSkThreads, 2)
     gemv_stream_kernel(const __grid_constant__ CUtensorMap tm0,
                        const __grid_constant__ CUtensorMap tm1, const SkParams p) {
     constexpr int NMAT = (MODE == kModeSwiglu) ? 2 : 1;
     constexpr int POS = Fmt<FMT>::kPos;
     constexpr int GPS = Fmt<FMT>::kGroups;
     constexpr int SCB = scb<FMT>();
-    constexpr int R = sk_ring<NMAT>();
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
 
+    const int R = p.R;
     const long long U = p.U;
     const int c = blockIdx.x;
     const long long u0 = U * c / p.nCTA, u1 = U * (c + 1) / p.nCTA;
-    const int nu = static_cast<int>(u1 - u0);
-    const int umax = static_cast<int>((U + p.nCTA - 1) / p.nCTA);
-    const SkLayout L = sk_layout<FMT, MT, NMAT>(p.SB, umax);
+    const int nitems = static_cast<int>(u1 - u0) * NMAT;
+    const int items_max = static_cast<int>((U + p.nCTA - 1) / p.nCTA) * NMAT;
+    const SkLayout L = sk_layout<FMT, MT>(p.SB, items_max, R);
     uint8_t *ring_w = smem;
     uint8_t *ring_s = smem + L.ring_s_off;
     uint8_t *act = smem + L.act_off;
     int *sq = reinterpret_cast<int *>(smem + L.sq_off);
+    float *xred = reinterpret_cast<float *>(smem + L.xred_off);
     float *sx = reinterpret_cast<float *>(smem + L.sx_off);
     float *red = reinterpret_cast<float *>(smem + L.red_off);
+    int *first_cnt = reinterpret_cast<int *>(smem + L.misc_off);
     float *slots = reinterpret_cast<float *>(smem + L.slots_off);
     uint64_t *full = reinterpret_cast<uint64_t *>(smem + L.bar_off);
     uint64_t *empty = full + R;
+    uint64_t *qbar1 = empty + R;  // the peers' partials of the row scale arrived
+    uint64_t *qbar2 = qbar1 + 1;  // the peers' int8 input and group sums arrived
 
+    const int C = static_cast<int>(cluster_nctarank());
+    const int rank = static_cast<int>(cluster_ctarank());
+    // This CTA's share of the 128-blocks of the padded input.
+    const int b_lo = L.GT * rank / C, b_hi = L.GT * (rank + 1) / C;
+    const int nown = b_hi - b_lo;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     if (tid == 0) {
         prefetch_tmap(&tm0);
@@ -248,155 +269,295 @@ __global__ void __launch_bounds__(kSkThreads, 1)
             mbar_init(&full[i], 1);
             mbar_init(&empty[i], 1);
         }
+        *first_cnt = 0;
+        mbar_init(qbar1, 1);
+        mbar_init(qbar2, 1);
+        mbar_arrive_expect_tx(qbar1, (C - 1) * MT * 8);
+        mbar_arrive_expect_tx(qbar2, MT * (L.GT - nown) * (128 + 16));
         fence_mbar_init();
     }
-    __syncthreads();
+    // Every CTA of the cluster has its barriers ready before any peer sends.
+    cluster_sync();
     pdl_launch_dependents();
 
     if (warp == 0) {
         // ---------------------------------------------------------- producer
+        // The whole warp walks the ring (one lane issues), so that no lane
+        // of it spins elsewhere while the copies are being issued.
+        cluster_arrive();  // sends nothing: the exit barrier's arrival
         if (!p.prefetch_ok) pdl_wait();
-        if (lane == 0) {
-            const uint64_t policy = l2_policy_evict_first();
-            for (int j = 0; j < nu; ++j) {
-                const int slot = j % R, round = j / R;
-                if (round > 0 && !mbar_wait_bounded(&empty[slot], (round - 1) & 1)) break;
-                const long long u = u0 + j;
-                const int rb = static_cast<int>(u / p.SB), sb = static_cast<int>(u % p.SB);
-                mbar_arrive_expect_tx(&full[slot], NMAT * (kTile + SCB));
-#pragma unroll
-                for (int mat = 0; mat < NMAT; ++mat) {
-                    tma_load_2d(ring_w + (slot * NMAT + mat) * kTile, mat ? &tm1 : &tm0,
-                                sb * kSBBytes, rb * 32, &full[slot], policy);
-                    const uint16_t *tsc = mat ? p.tsc1 : p.tsc0;
-                    bulk_copy_g2s(ring_s + (slot * NMAT + mat) * SCB,
-                                  reinterpret_cast<const uint8_t *>(tsc) + u * SCB, SCB, &full[slot],
-                                  policy);
+        const uint64_t policy = l2_policy_evict_first();
+        // Positions advance incrementally: no division inside the loop.
+        int slot = 0, round = 0, mat = 0;
+        int rb = static_cast<int>(u0 / p.SB), sb = static_cast<int>(u0 % p.SB);
+        const uint8_t *sc_unit[2] = {reinterpret_cast<const uint8_t *>(p.tsc0) + u0 * SCB,
+                                     reinterpret_cast<const uint8_t *>(p.tsc1) + u0 * SCB};
+        for (int j = 0; j < nitems; ++j) {
+            if (round > 0 &&
+                !__all_sync(0xffffffffu, mbar_wait_bounded(&empty[slot], (round - 1) & 1)))
+                break;
+            if (lane == 0) {
+                mbar_arrive_expect_tx(&full[slot], kTile + SCB);
+                tma_load_2d(ring_w + slot * kTile, mat ? &tm1 : &tm0, sb * kSBBytes, rb * 32,
+                            &full[slot], policy);
+                bulk_copy_g2s(ring_s + slot * SCB, sc_unit[mat], SCB, &full[slot], policy);
+            }
+            __syncwarp();
+            if (NMAT == 2 && mat == 0) {
+                mat = 1;
+            } else {
+                mat = 0;
+                sc_unit[0] += SCB;
+                sc_unit[1] += SCB;
+                if (++sb == p.SB) {
+                    sb = 0;
+                    ++rb;
                 }
+            }
+            if (++slot == R) {
+                slot = 0;
+                ++round;
             }
         }
     } else {
         // ---------------------------------------------------------- consumers
         const int cw = warp - 1, ctid = tid - 32;
+        const int rb_lo = static_cast<int>(u0 / p.SB);
+        const int rb_hi = static_cast<int>((u1 - 1) / p.SB);
+        // A cut first row block is published (its end is here), a cut last
+        // row block is finished here (its start is here).
+        const bool publish = static_cast<long long>(rb_lo) * p.SB < u0;
+        const bool combine = static_cast<long long>(rb_hi + 1) * p.SB > u1;
+        const int n_first = publish ? static_cast<int>((static_cast<long long>(rb_lo + 1) * p.SB - u0) * NMAT) : 0;
         pdl_wait();
+        // Residual of the first row block this warp finishes, fetched early.
+        float res0[MT];
+#pragma unroll
+        for (int m = 0; m < MT; ++m) {
+            res0[m] = 0.0f;
+            const int n = (rb_lo + cw) * 32 + lane;
+            if (MODE == kModeGemv && p.residual && rb_lo + cw <= rb_hi && n < p.N && m < p.M)
+                res0[m] = __ldcg(p.residual + static_cast<int64_t>(m) * p.ldo + n);
+        }
         const bool rotate = (p.qflags & TERN_QUANT_FWHT128) != 0;
         const bool rms = (p.qflags & TERN_QUANT_RMSNORM) != 0;
-        const int nb = (p.K + 127) / 128;    // blocks holding input
-        const int nbpad = L.Kpad / 128;      // blocks of the padded activation
-        // pass 1: max |x| (or |H x|) and sum x^2 per token row
+
+        // pass 1: loads first (kSkKeep blocks per warp in flight), then the
+        // rotation, max |.| and sum x^2 of this CTA's blocks
+        float v[MT][kSkKeep][4];
+        float amax[MT], ss[MT];
+#pragma unroll
         for (int m = 0; m < MT; ++m) {
-            float amax = 0.0f, ss = 0.0f;
-            if (m < p.M) {
-                for (int b = cw; b < nb; b += kSkConsumers) {
-                    const int k = 128 * b + 4 * lane;
-                    float r[4] = {0.0f, 0.0f, 0.0f, 0.0f};
-                    const float *src = p.x + static_cast<int64_t>(m) * p.ldx + k;
-                    if (k + 4 <= p.K) {
-                        const float4 v = *reinterpret_cast<const float4 *>(src);
-                        r[0] = v.x;
-                        r[1] = v.y;
-                        r[2] = v.z;
-                        r[3] = v.w;
-                    } else {
-                        for (int e = 0; e < 4 && k + e < p.K; ++e) r[e] = src[e];
-                    }
-                    ss += fmaf(r[3], r[3], fmaf(r[2], r[2], fmaf(r[1], r[1], r[0] * r[0])));
-                    if (rotate) fwht128_warp(r, lane);
-                    amax = fmaxf(amax, fmaxf(fmaxf(fabsf(r[0]), fabsf(r[1])), fmaxf(fabsf(r[2]), fabsf(r[3]))));
+            amax[m] = 0.0f;
+            ss[m] = 0.0f;
+#pragma unroll
+            for (int j = 0; j < kSkKeep; ++j) {
+                const int b = b_lo + cw + kSkConsumers * j;
+                if (b < b_hi) {
+                    load_block(p, m, b, lane, v[m][j]);
+                } else {
+                    v[m][j][0] = v[m][j][1] = v[m][j][2] = v[m][j][3] = 0.0f;
                 }
             }
-            amax = warp_max(amax);
-            ss = warp_sum(ss);
+        }
+#pragma unroll
+        for (int m = 0; m < MT; ++m)
+#pragma unroll
+            for (int j = 0; j < kSkKeep; ++j) {
+                if (b_lo + cw + kSkConsumers * j >= b_hi) continue;
+                ss[m] += sumsq4(v[m][j]);
+                if (rotate) fwht128_warp(v[m][j], lane);
+                amax[m] = fmaxf(amax[m], amax4(v[m][j]));
+            }
+        for (int b = b_lo + cw + kSkConsumers * kSkKeep; b < b_hi; b += kSkConsumers) {
+#pragma unroll
+            for (int m = 0; m < MT; ++m) {
+                float r[4];
+                load_block(p, m, b, lane, r);
+                ss[m] += sumsq4(r);
+                if (rotate) fwht128_warp(r, lane);
+                amax[m] = fmaxf(amax[m], amax4(r));
+            }
+        }
+#pragma unroll
+        for (int m = 0; m < MT; ++m) {
+            const float a = warp_max(amax[m]);
+            const float s = warp_sum(ss[m]);
             if (lane == 0) {
-                red[(cw * MT + m) * 2 + 0] = amax;
-                red[(cw * MT + m) * 2 + 1] = ss;
+                red[(cw * MT + m) * 2 + 0] = a;
+                red[(cw * MT + m) * 2 + 1] = s;
             }
         }
         warpgroup_sync_n(kSkBar, kSkConsumers * 32);
         if (ctid < MT) {
+            // this CTA's share (fixed warp order): kept here, sent to the peers
             const int m = ctid;
-            float amax = 0.0f, ss = 0.0f;
+            float a = 0.0f, s = 0.0f;
             for (int w = 0; w < kSkConsumers; ++w) {
-                amax = fmaxf(amax, red[(w * MT + m) * 2 + 0]);
-                ss += red[(w * MT + m) * 2 + 1];
+                a = fmaxf(a, red[(w * MT + m) * 2 + 0]);
+                s += red[(w * MT + m) * 2 + 1];
             }
-            float inv = 0.0f, s = 0.0f;
-            if (amax > 0.0f) {
-                inv = __fdiv_rn(127.0f, amax);
-                s = __fdiv_rn(amax, 127.0f);
-                if (rotate) s = __fmul_rn(s, kInvSqrt128);
-            }
-            if (rms) s = s / sqrtf(ss / static_cast<float>(p.K) + 1e-6f);
-            sx[m] = s;
-            sx[MT + m] = inv;
+            xred[(rank * MT + m) * 2 + 0] = a;
+            xred[(rank * MT + m) * 2 + 1] = s;
+            for (int q = 0; q < C; ++q)
+                if (q != rank)
+                    st_async_v2f32(map_shared_rank(xred + (rank * MT + m) * 2, q), a, s,
+                                   map_shared_rank(qbar1, q));
         }
         warpgroup_sync_n(kSkBar, kSkConsumers * 32);
-        // pass 2: int8 codes of every block and the per-group sums
-        for (int job = cw; job < MT * nbpad; job += kSkConsumers) {
-            const int m = job / nbpad, b = job % nbpad;
-            const int k = 128 * b + 4 * lane;
-            float r[4] = {0.0f, 0.0f, 0.0f, 0.0f};
-            if (m < p.M && k < p.K) {
-                const float *src = p.x + static_cast<int64_t>(m) * p.ldx + k;
-                if (k + 4 <= p.K) {
-                    const float4 v = *reinterpret_cast<const float4 *>(src);
-                    r[0] = v.x;
-                    r[1] = v.y;
-                    r[2] = v.z;
-                    r[3] = v.w;
-                } else {
-                    for (int e = 0; e < 4 && k + e < p.K; ++e) r[e] = src[e];
-                }
+        const bool ok1 = mbar_wait_cluster_bounded(qbar1, 0);
+        // Row scale from the cluster's shares (same order in every CTA).
+        float inv[MT];
+#pragma unroll
+        for (int m = 0; m < MT; ++m) {
+            float a = 0.0f, s = 0.0f;
+            for (int q = 0; q < C; ++q) {
+                const bool have = ok1 || q == rank;
+                a = fmaxf(a, have ? xred[(q * MT + m) * 2 + 0] : 0.0f);
+                s += have ? xred[(q * MT + m) * 2 + 1] : 0.0f;
             }
-            if (rotate) fwht128_warp(r, lane);
-            const float inv = sx[MT + m];
+            float iv = 0.0f, sc = 0.0f;
+            if (a > 0.0f) {
+                iv = __fdiv_rn(127.0f, a);
+                sc = __fdiv_rn(a, 127.0f);
+                if (rotate) sc = __fmul_rn(sc, kInvSqrt128);
+            }
+            if (rms) sc = sc / sqrtf(s / static_cast<float>(p.K) + 1e-6f);
+            inv[m] = iv;
+            if (ctid == 0) sx[m] = sc;
+        }
+
+        // pass 2: int8 codes and group sums of this CTA's blocks, written
+        // here, then one bulk copy of the share to each peer
+        auto quant_block = [&](int m, int b, const float (&r)[4]) {
             uint32_t packed = 0;
             int qsum = 0;
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
                 int qi = 0;
-                if (k + e < p.K && inv > 0.0f) {
-                    qi = __float2int_rn(__fmul_rn(r[e], inv));
+                if (inv[m] > 0.0f) {
+                    qi = __float2int_rn(__fmul_rn(r[e], inv[m]));
                     qi = max(-127, min(127, qi));
                 }
                 qsum += qi;
                 packed |= (static_cast<uint32_t>(qi) & 0xffu) << (8 * e);
             }
-            *reinterpret_cast<uint32_t *>(act + m * L.Kpad + k) = packed;
             qsum = warp_sum_int(qsum);
-            if (lane == 0) sq[m * L.GT + b] = qsum;
+            *reinterpret_cast<uint32_t *>(act + m * L.Kpad + 128 * b + 4 * lane) = packed;
+            if (lane == 0) sq[(m * L.GT + b) * 4] = qsum;
+        };
+#pragma unroll
+        for (int m = 0; m < MT; ++m)
+#pragma unroll
+            for (int j = 0; j < kSkKeep; ++j) {
+                const int b = b_lo + cw + kSkConsumers * j;
+                if (b < b_hi) quant_block(m, b, v[m][j]);
+            }
+        for (int b = b_lo + cw + kSkConsumers * kSkKeep; b < b_hi; b += kSkConsumers) {
+#pragma unroll
+            for (int m = 0; m < MT; ++m) {
+                float r[4];
+                load_block(p, m, b, lane, r);
+                if (rotate) fwht128_warp(r, lane);
+                quant_block(m, b, r);
+            }
         }
+        fence_proxy_async_smem();  // the share is read by the bulk copies
         warpgroup_sync_n(kSkBar, kSkConsumers * 32);
+        if (ctid == 0 && nown > 0) {
+            for (int q = 0; q < C; ++q) {
+                if (q == rank) continue;
+                const uint32_t bar = map_shared_rank(qbar2, q);
+                for (int m = 0; m < MT; ++m) {
+                    uint8_t *a = act + m * L.Kpad + 128 * b_lo;
+                    int *g = sq + (m * L.GT + b_lo) * 4;
+                    bulk_copy_s2cluster(map_shared_rank(a, q), a, 128 * nown, bar);
+                    bulk_copy_s2cluster(map_shared_rank(g, q), g, 16 * nown, bar);
+                }
+            }
+        }
+        const bool ok2 = mbar_wait_cluster_bounded(qbar2, 0);
+        // Everything sent to this CTA has landed: its exit no longer waits
+        // on it (and the peers' copies out of their shared memory are done).
+        cluster_arrive();
 
-        // units, round-robin over the consumer warps
-        for (int j = cw; j < nu; j += kSkConsumers) {
-            const int slot = j % R;
-            const bool ok = __all_sync(0xffffffffu, mbar_wait_bounded(&full[slot], (j / R) & 1));
-            float yacc[NMAT][MT];
+        // items, round-robin over the consumer warps; the slot is handed back
+        // as soon as the item sits in registers.  Slot, phase and superblock
+        // advance incrementally (R >= kSkConsumers: at most one wrap a step).
+        int slot = cw, phase = 0;
+        int sb = static_cast<int>((u0 + cw / NMAT) % p.SB);
+        for (int j = cw; j < nitems; j += kSkConsumers) {
+            const bool ok =
+                ok2 && __all_sync(0xffffffffu, mbar_wait_bounded(&full[slot], phase));
+            float yacc[MT];
             if (ok) {
-                const long long u = u0 + j;
-                const int sb = static_cast<int>(u % p.SB);
-                sk_unit<FMT, MT, NMAT>(ring_w + slot * NMAT * kTile, ring_s + slot * NMAT * SCB, lane,
-                                       act + sb * POS, L.Kpad, sq + sb * GPS, L.GT, yacc);
+                uint32_t words[32];
+                const uint8_t *wt = ring_w + slot * kTile + lane * kSBBytes;
+                const int rsw = lane & 7;
+#pragma unroll
+                for (int cc = 0; cc < 8; ++cc) {
+                    const uint4 wv = lds128(wt + ((cc ^ rsw) << 4));
+                    words[4 * cc + 0] = wv.x;
+                    words[4 * cc + 1] = wv.y;
+                    words[4 * cc + 2] = wv.z;
+                    words[4 * cc + 3] = wv.w;
+                }
+                float sc[GPS];
+                const uint16_t *st =
+                    reinterpret_cast<const uint16_t *>(ring_s + slot * SCB) + lane * GPS;
+#pragma unroll
+                for (int g = 0; g < GPS; ++g) sc[g] = __half2float(__ushort_as_half(st[g]));
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&empty[slot]);
+                sk_item<FMT, MT>(words, sc, act + sb * POS, L.Kpad, sq + sb * GPS * 4, L.GT, yacc);
             } else {
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&empty[slot]);
 #pragma unroll
-                for (int mat = 0; mat < NMAT; ++mat)
-#pragma unroll
-                    for (int m = 0; m < MT; ++m) yacc[mat][m] = 0.0f;
+                for (int m = 0; m < MT; ++m) yacc[m] = 0.0f;
             }
 #pragma unroll
-            for (int mat = 0; mat < NMAT; ++mat)
+            for (int m = 0; m < MT; ++m) slots[(j * MT + m) * 32 + lane] = yacc[m];
+            slot += kSkConsumers;
+            if (slot >= R) {
+                slot -= R;
+                phase ^= 1;
+            }
+            sb += kSkConsumers / NMAT;
+            while (sb >= p.SB) sb -= p.SB;
+            if (j < n_first) {
+                // The last warp to finish an item of the cut first row block
+                // publishes that row block's partial (value and tag in one
+                // 64-bit store) for the CTA holding its start.
+                __syncwarp();
+                int done = 0;
+                if (lane == 0) {
+                    __threadfence_block();
+                    done = atomicAdd(first_cnt, 1);
+                }
+                done = __shfl_sync(0xffffffffu, done, 0);
+                if (done == n_first - 1) {
+                    __threadfence_block();
+                    const long long ue = static_cast<long long>(rb_lo + 1) * p.SB;
 #pragma unroll
-                for (int m = 0; m < MT; ++m) slots[((j * NMAT + mat) * MT + m) * 32 + lane] = yacc[mat][m];
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&empty[slot]);
+                    for (int mat = 0; mat < NMAT; ++mat)
+#pragma unroll
+                        for (int m = 0; m < MT; ++m) {
+                            float s = 0.0f;
+                            for (long long uu = u0; uu < ue; ++uu)
+                                s += slots[(((uu - u0) * NMAT + mat) * MT + m) * 32 + lane];
+                            st_relaxed_gpu_u64(p.ws_tag + tag_index<NMAT, MT>(rb_lo, mat, m, lane),
+                                               (1ull << 32) | __float_as_uint(s));
+                        }
+                }
+            }
         }
         warpgroup_sync_n(kSkBar, kSkConsumers * 32);
 
-        // row blocks of this range: sum units in order; finish or combine
-        const int rb_lo = static_cast<int>(u0 / p.SB);
-        const int rb_hi = static_cast<int>((u1 - 1) / p.SB);
-        for (int rb = rb_lo + cw; rb <= rb_hi; rb += kSkConsumers) {
+        // row blocks of this range: sum units in order; finish
+        int i = 0;
+        for (int rb = rb_lo + cw; rb <= rb_hi; rb += kSkConsumers, ++i) {
+            if (rb == rb_lo && publish) continue;
             const long long ua = max(u0, static_cast<long long>(rb) * p.SB);
             const long long ub = min(u1, static_cast<long long>(rb + 1) * p.SB);
             float tot[NMAT][MT];
@@ -409,77 +570,96 @@ __global__ void __launch_bounds__(kSkThreads, 1)
                         s += slots[(((u - u0) * NMAT + mat) * MT + m) * 32 + lane];
                     tot[mat][m] = s;
                 }
-            const bool lower_cut = static_cast<long long>(rb) * p.SB < u0;
-            const bool upper_cut = static_cast<long long>(rb + 1) * p.SB > u1;
-            bool finish_here = true;
-            if (lower_cut || upper_cut) {
-                const int side = lower_cut ? 1 : 0;  // 0: this CTA holds the row block's start
+            if (rb == rb_hi && combine) {
+                // this CTA holds the start: add the partial the next CTA
+                // published (bounded wait), then clear it for the next call
 #pragma unroll
                 for (int mat = 0; mat < NMAT; ++mat)
 #pragma unroll
-                    for (int m = 0; m < MT; ++m)
-                        p.ws_part[((((static_cast<int64_t>(rb) * 2 + side) * NMAT + mat) * MT + m) * 32) +
-                                  lane] = tot[mat][m];
-                __threadfence();
-                __syncwarp();
-                int old = 0;
-                if (lane == 0) old = atomicAdd(&p.ws_cnt_end[-1 - rb], 1);
-                old = __shfl_sync(0xffffffffu, old, 0);
-                finish_here = (old == 1);
-                if (finish_here) {
-                    __threadfence();
-#pragma unroll
-                    for (int mat = 0; mat < NMAT; ++mat)
-#pragma unroll
-                        for (int m = 0; m < MT; ++m) {
-                            const int64_t base = (((static_cast<int64_t>(rb) * 2) * NMAT + mat) * MT + m) * 32 + lane;
-                            const float lo = __ldcg(p.ws_part + base);
-                            const float hi = __ldcg(p.ws_part + base + static_cast<int64_t>(NMAT) * MT * 32);
-                            tot[mat][m] = lo + hi;
+                    for (int m = 0; m < MT; ++m) {
+                        unsigned long long *t = p.ws_tag + tag_index<NMAT, MT>(rb, mat, m, lane);
+                        unsigned long long w = ld_relaxed_gpu_u64(t);
+                        if ((w >> 32) == 0) {
+                            const long long start = clock64();
+                            while (((w = ld_relaxed_gpu_u64(t)) >> 32) == 0) {
+                                if (clock64() - start > kWaitBudgetCycles) {
+                                    atomicExch(&g_device_error, kErrTmaTimeout);
+                                    break;
+                                }
+                            }
                         }
-                    if (lane == 0) p.ws_cnt_end[-1 - rb] = 0;
-                }
+                        tot[mat][m] = tot[mat][m] + __uint_as_float(static_cast<uint32_t>(w));
+                        st_relaxed_gpu_u64(t, 0ull);
+                    }
             }
-            if (!finish_here) continue;
             const int n = rb * 32 + lane;
             if (n >= p.N) continue;
 #pragma unroll
             for (int m = 0; m < MT; ++m) {
                 if (m >= p.M) continue;
                 const int64_t o = static_cast<int64_t>(m) * p.ldo + n;
-                float v;
+                float val;
                 if (MODE == kModeGemv) {
-                    v = sx[m] * tot[0][m];
-                    if (p.residual) v += p.residual[o];
+                    val = sx[m] * tot[0][m];
+                    if (p.residual) val += (i == 0) ? res0[m] : p.residual[o];
                 } else {
                     const float g = sx[m] * tot[0][m];
-                    const float u = sx[m] * tot[NMAT - 1][m];
-                    v = g * (1.0f / (1.0f + expf(-g))) * u;
+                    const float up = sx[m] * tot[NMAT - 1][m];
+                    val = g * (1.0f / (1.0f + expf(-g))) * up;
                 }
-                p.out[o] = v;
+                p.out[o] = val;
             }
         }
+        if (!ok2) mbar_wait_cluster_bounded(qbar2, 0);  // let late copies land before exit
     }
-    __syncthreads();
+    // No CTA leaves while a peer of its cluster may still copy into it.
+    cluster_wait();
 }
 
 constexpr int kMaxDevices = 64;
 
+// Cluster size for the input quantisation: the largest of {4, 2} whose
+// clusters keep at least 97% of the SMs busy with one CTA each, else 1.
+// Returns the size and (in *ncta) the CTAs that are resident at once.
+template <typename Kern>
+int choose_cluster(Kern kern, int num_sms, int *ncta) {
+    for (int C : {4, 2}) {
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3((num_sms / C) * C, 1, 1);
+        cfg.blockDim = dim3(kSkThreads, 1, 1);
+        cfg.dynamicSmemBytes = 200 * 1024;  // one CTA per SM
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = C;
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        int nclusters = 0;
+        if (cudaOccupancyMaxActiveClusters(&nclusters, kern, &cfg) != cudaSuccess) {
+            (void)cudaGetLastError();
+            continue;
+        }
+        const int n = nclusters * C;
+        if (n * 100 >= num_sms * 97) {
+            *ncta = n < num_sms ? n : num_sms;
+            return C;
+        }
+    }
+    *ncta = num_sms;
+    return 1;
+}
+
 template <int FMT, int MT, int MODE>
 cudaError_t launch_sk(const StreamLaunch &S, cudaStream_t s, const char **why) {
     constexpr int NMAT = (MODE == kModeSwiglu) ? 2 : 1;
-    static int smem_set[kMaxDevices] = {0};
+    static int plan_c[kMaxDevices] = {0}, plan_n[kMaxDevices] = {0};
     SkParams p = {};
     p.N = S.N;
     p.K = S.K;
-    p.G = static_cast<int>(ceil_div(S.K, 128));
     p.SB = static_cast<int>(ceil_div(S.row_bytes, kSBBytes));
     p.RB = static_cast<int>(ceil_div(S.N, 32));
     p.U = static_cast<long long>(p.RB) * p.SB;
-    long long ncta = p.U / p.SB;  // every range holds >= SB units: a row block meets <= 2 ranges
-    if (ncta > S.num_sms) ncta = S.num_sms;
-    if (ncta < 1) ncta = 1;
-    p.nCTA = static_cast<int>(ncta);
     p.M = S.M;
     p.prefetch_ok = S.prefetch_ok;
     p.qflags = S.qflags;
@@ -490,12 +670,31 @@ cudaError_t launch_sk(const StreamLaunch &S, cudaStream_t s, const char **why) {
     p.residual = S.residual;
     p.out = S.out;
     p.ldo = S.ldo;
-    // Partial sums from the start of the workspace, counters from its end:
-    // every call finds counter rb at the same place, whatever its own size.
-    p.ws_part = static_cast<float *>(S.workspace);
-    p.ws_cnt_end = reinterpret_cast<int *>(static_cast<char *>(S.workspace) + (S.ws_bytes & ~size_t(3)));
-    const int umax = static_cast<int>((p.U + p.nCTA - 1) / p.nCTA);
-    const SkLayout L = sk_layout<FMT, MT, NMAT>(p.SB, umax);
+    p.ws_tag = static_cast<unsigned long long *>(S.workspace);
+
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+    auto kern = gemv_stream_kernel<FMT, MT, MODE>;
+    if (!plan_c[dev]) {
+        e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
+        if (e != cudaSuccess) return e;
+        plan_c[dev] = choose_cluster(kern, S.num_sms, &plan_n[dev]);
+    }
+    // every range holds >= SB units, so a row block meets at most 2 ranges
+    long long want = p.U / p.SB;
+    if (want > plan_n[dev]) want = plan_n[dev];
+    if (want < 1) want = 1;
+    int C = plan_c[dev];
+    while (C > 1 && want < C) C /= 2;
+    p.nCTA = static_cast<int>((want / C) * C);
+    const int items_max = static_cast<int>((p.U + p.nCTA - 1) / p.nCTA) * NMAT;
+    // ring depth: as many slots as fit the two-CTAs-per-SM budget
+    int R = kSkMaxRing;
+    while (R > kSkMinRing && sk_layout<FMT, MT>(p.SB, items_max, R).total > kSkSmemBudget) --R;
+    p.R = R;
+    const SkLayout L = sk_layout<FMT, MT>(p.SB, items_max, R);
     if (L.total > 227 * 1024) {
         *why = "shared memory plan of the streamed kernel exceeds 227 KB";
         return cudaErrorInvalidValue;
@@ -506,26 +705,21 @@ cudaError_t launch_sk(const StreamLaunch &S, cudaStream_t s, const char **why) {
         *why = "cuTensorMapEncodeTiled failed or is unavailable";
         return cudaErrorInvalidValue;
     }
-    int dev = 0;
-    cudaError_t e = cudaGetDevice(&dev);
-    if (e != cudaSuccess) return e;
-    if (dev >= 0 && dev < kMaxDevices && !smem_set[dev]) {
-        e = cudaFuncSetAttribute(gemv_stream_kernel<FMT, MT, MODE>,
-                                 cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
-        if (e != cudaSuccess) return e;
-        smem_set[dev] = 1;
-    }
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(p.nCTA, 1, 1);
     cfg.blockDim = dim3(kSkThreads, 1, 1);
     cfg.dynamicSmemBytes = L.total;
     cfg.stream = s;
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[0].val.programmaticStreamSerializationAllowed = 1;
+    attr[1].id = cudaLaunchAttributeClusterDimension;
+    attr[1].val.clusterDim.x = C;
+    attr[1].val.clusterDim.y = 1;
+    attr[1].val.clusterDim.z = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    e = cudaLaunchKernelEx(&cfg, gemv_stream_kernel<FMT, MT, MODE>, tm0, tm1, p);
+    cfg.numAttrs = C > 1 ? 2 : 1;
+    e = cudaLaunchKernelEx(&cfg, kern, tm0, tm1, p);
     if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }

@@ -103,6 +103,25 @@ cudaError_t launch_act_stats(const float *x, int M, int K, int ldx, float *stats
                              cudaStream_t s);
 cudaError_t read_clear_device_error(int *value, cudaStream_t s);
 
+// 2-D uint8 tensor map with 128-byte swizzle (tern_gemv.cu).
+bool make_u8_tmap_2d(CUtensorMap *map, const void *base, uint64_t inner, uint64_t rows,
+                     uint64_t stride, uint32_t box_inner, uint32_t box_rows);
+
+// ---------------------------------------------------------------- prefill GEMM
+struct GemmLaunch {
+    int fmt;
+    int N, K, M;
+    int64_t row_bytes, row_stride;
+    const void *packed;
+    const uint16_t *scales;
+    const int8_t *q;
+    int ldq;
+    const float *s_x;
+    float *y;
+    int ldy;
+};
+cudaError_t launch_gemm(const GemmLaunch &L, cudaStream_t s, const char **why);
+
 // Sets the message tern_last_error() returns on the calling host thread.
 tern_status set_last_error(tern_status s, const char *message);
 

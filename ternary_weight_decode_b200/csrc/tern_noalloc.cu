@@ -1,7 +1,7 @@
 // tern_noalloc.cu -- tern_gemv_streamed for callers that cannot allocate
-// device memory: the streamed kernel's scratch (fp32 partial sums of the row
-// blocks cut between two CTAs, and their arrival counters) lives in a fixed
-// array that the library itself holds on every device that loads it.
+// device memory: the streamed kernel's scratch (partial sums of the row
+// blocks cut between two CTAs) lives in a fixed array that the library
+// itself holds on every device that loads it.
 #include <stdio.h>
 
 #include <mutex>
@@ -12,8 +12,8 @@
 namespace {
 
 // Held on every device that loads the library, for as long as the process
-// runs.  Shared by every call on that device; each call clears the counters
-// it uses, the partial sums need no clearing.
+// runs.  Shared by every call on that device; each call clears the part it
+// uses before its kernel runs.
 static __device__ __align__(256) unsigned char g_noalloc_scratch[TERN_NOALLOC_SCRATCH_BYTES];
 
 constexpr int kMaxDevices = 64;
@@ -67,11 +67,9 @@ tern_status tern_gemv_streamed_noalloc(const tern_matrix *W, const float *x, int
                  cudaGetErrorString(e));
         return tern::set_last_error(TERN_ECUDA, msg);
     }
-    // The counters of this call's row blocks sit at the end of the array;
-    // clear them, whatever an earlier (possibly failed) call left there.
-    const size_t counters = static_cast<size_t>(tern::ceil_div(W->N, 32)) * sizeof(int);
-    e = cudaMemsetAsync(static_cast<unsigned char *>(scratch) + bytes - counters, 0, counters,
-                        static_cast<cudaStream_t>(stream));
+    // The kernel expects the scratch it uses to start at zero; clear it,
+    // whatever an earlier (possibly failed) call left there.
+    e = cudaMemsetAsync(scratch, 0, need, static_cast<cudaStream_t>(stream));
     if (e != cudaSuccess) {
         char msg[256];
         snprintf(msg, sizeof(msg), "tern_gemv_streamed_noalloc: clearing the counters: %s",

@@ -175,6 +175,22 @@ __device__ __forceinline__ uint64_t smem_desc_noswizzle(uint32_t saddr, uint32_t
            (static_cast<uint64_t>((sbo >> 4) & 0x3FFFu) << 32) | (1ull << 46);
 }
 
+// Shared-memory matrix descriptor, K-major with 128-byte swizzle: rows of
+// 128 bytes (128 8-bit K elements), 16-byte chunk c of row r stored at chunk
+// c ^ (r % 8) (the pattern TMA writes with CU_TENSOR_MAP_SWIZZLE_128B), 8-row
+// groups 1024 bytes apart (SBO); the tile base 1024-byte aligned.  Steps of
+// 32 K elements inside the 128-byte row advance the start address by 32.
+//   layout type [61,64) = 2 (128-byte swizzle), LBO unused (16).
+__device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t saddr) {
+    return static_cast<uint64_t>((saddr >> 4) & 0x3FFFu) | (static_cast<uint64_t>(1u) << 16) |
+           (static_cast<uint64_t>(1024u >> 4) << 32) | (1ull << 46) | (2ull << 61);
+}
+
+// Byte offset of element (r, k) (k < 128) in a 128-byte-swizzled K-major tile.
+__host__ __device__ constexpr uint32_t sw128_offset(uint32_t r, uint32_t k) {
+    return r * 128u + ((((k >> 4) ^ (r & 7u)) & 7u) << 4) + (k & 15u);
+}
+
 // ---------------------------------------------------------------- MMA
 // D[tmem] (+)= A[tmem] * B[smem]^T, issued by one thread.
 __device__ __forceinline__ void mma_i8_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,

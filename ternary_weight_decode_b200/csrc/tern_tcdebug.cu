@@ -2,8 +2,9 @@
 // computes D = A * B^T for a 128 x K int8 A and an N x K int8 B, with A taken
 // from tensor memory (written by tcgen05.st, as the decode kernels write
 // their decoded operand) or from shared memory, B from shared memory in the
-// no-swizzle core-matrix layout.  Used by the tests to pin the descriptor
-// encodings against a plain integer product.
+// no-swizzle core-matrix layout -- or (mode 2) both from shared memory in the
+// 128-byte-swizzled K-major layout the prefill GEMM uses.  Used by the tests
+// to pin the descriptor encodings against a plain integer product.
 #include "tern_common.cuh"
 #include "tern_internal.h"
 #include "tern_tc.cuh"
@@ -29,11 +30,19 @@ __global__ void __launch_bounds__(128)
         mbar_init(&bar, 1);
         fence_mbar_init();
     }
-    for (int idx = tid; idx < N * K; idx += 128)
-        sb[core_offset(idx / K, idx % K, N)] = static_cast<uint8_t>(B[idx]);
+    const bool sw = a_in_smem == 2;
+    // mode 2: 128-K blocks, each an [rows][128 B] swizzled tile
+    for (int idx = tid; idx < N * K; idx += 128) {
+        const int n = idx / K, k = idx % K;
+        sb[sw ? (k >> 7) * N * 128 + sw128_offset(n, k & 127) : core_offset(n, k, N)] =
+            static_cast<uint8_t>(B[idx]);
+    }
     if (a_in_smem)
-        for (int idx = tid; idx < 128 * K; idx += 128)
-            sa[core_offset(idx / K, idx % K, 128)] = static_cast<uint8_t>(A[idx]);
+        for (int idx = tid; idx < 128 * K; idx += 128) {
+            const int r = idx / K, k = idx % K;
+            sa[sw ? (k >> 7) * 128 * 128 + sw128_offset(r, k & 127) : core_offset(r, k, 128)] =
+                static_cast<uint8_t>(A[idx]);
+        }
     fence_proxy_async_smem();
     tc_fence_before_sync();
     __syncthreads();
@@ -59,6 +68,13 @@ __global__ void __launch_bounds__(128)
         tc_fence_after_sync();
         const uint32_t idesc = idesc_i8(128, N, a_signed, b_signed);
         for (int ks = 0; ks < K / 32; ++ks) {
+            if (sw) {
+                const int kb = ks >> 2, kk = (ks & 3) * 32;
+                const uint64_t bd = smem_desc_sw128(smem_u32(sb) + kb * N * 128 + kk);
+                const uint64_t ad = smem_desc_sw128(smem_u32(sa) + kb * 128 * 128 + kk);
+                mma_i8_ss(tbase + kDbgDCol, ad, bd, idesc, ks > 0);
+                continue;
+            }
             const uint64_t bd = smem_desc_noswizzle(smem_u32(sb) + ks * 2 * (N / 8) * 128,
                                                     (N / 8) * 128, 128);
             if (a_in_smem) {

@@ -88,6 +88,7 @@ def lib() -> ctypes.CDLL:
                 "tern_gateup_swiglu_streamed": (ctypes.c_int, [pm, pm, p, i32, i32, i32, p, i32, p, sz,
                                                                p]),
                 "tern_gemv_streamed_noalloc": (ctypes.c_int, [pm, p, i32, i32, i32, p, p, i32, p]),
+                "tern_gemm": (ctypes.c_int, [pm, p, i32, p, i32, p, i32, p]),
                 "tern_gemv_fused": (ctypes.c_int, [pm, p, i32, p, i32, i32, i32, p, p, i32, p, i32, p]),
                 "tern_gateup_swiglu_fused": (ctypes.c_int, [pm, pm, p, i32, p, i32, i32, i32, p, i32,
                                                             p, i32, p]),
@@ -239,6 +240,17 @@ def tern_gemv(W: TernMatrix, q: torch.Tensor, s_x: torch.Tensor, y: torch.Tensor
                            _ptr(y), y.stride(0), _stream(stream)), "tern_gemv")
 
 
+def tern_gemm(W: TernMatrix, q: torch.Tensor, s_x: torch.Tensor, y: torch.Tensor, M: int | None = None,
+              stream=None):
+    """Prefill GEMM: y [M, N] = s_x * (group-scaled W q) on the tensor cores."""
+    M = q.shape[0] if M is None else M
+    assert q.dtype == torch.int8 and q.stride(1) == 1 and y.dtype == torch.float32
+    s = W.struct()
+    _check(lib().tern_gemm(ctypes.byref(s), _ptr(q), q.stride(0), _ptr(s_x), M, _ptr(y), y.stride(0),
+                           _stream(stream)),
+           "tern_gemm")
+
+
 def tern_gateup_swiglu(Wg: TernMatrix, Wu: TernMatrix, q: torch.Tensor, s_x: torch.Tensor,
                        h: torch.Tensor, M: int | None = None, stream=None):
     M = q.shape[0] if M is None else M
@@ -300,12 +312,14 @@ def tern_gateup_swiglu_fused(Wg: TernMatrix, Wu: TernMatrix, x: torch.Tensor,
                                           _stream(stream)), "tern_gateup_swiglu_fused")
 
 
-def tern_debug_mma_i8(A: torch.Tensor, B: torch.Tensor, D: torch.Tensor, a_in_smem: bool = False,
+def tern_debug_mma_i8(A: torch.Tensor, B: torch.Tensor, D: torch.Tensor, a_in_smem: int = 0,
                       a_signed: bool = True, b_signed: bool = True, stream=None):
-    """D int32 [128, N] = A [128, K] . B [N, K]^T on the tensor cores (test hook)."""
+    """D int32 [128, N] = A [128, K] . B [N, K]^T on the tensor cores (test hook).
+    a_in_smem: 0 A in tensor memory, 1 A in shared memory, 2 both operands in
+    the 128-byte-swizzled layout."""
     K = A.shape[1]
     N = B.shape[0]
-    _check(lib().tern_debug_mma_i8(1 if a_in_smem else 0, _ptr(A), 1 if a_signed else 0, _ptr(B),
+    _check(lib().tern_debug_mma_i8(int(a_in_smem), _ptr(A), 1 if a_signed else 0, _ptr(B),
                                    1 if b_signed else 0, _ptr(D), K, N, _stream(stream)),
            "tern_debug_mma_i8")
 

@@ -118,3 +118,15 @@ def test_act_quant_rejects_unknown_flags():
     st = lib.act_quant_fwht(ctypes.c_void_p(4096), 1, 1, 256, 256, 0, 2, ctypes.c_void_p(4096), 256,
                             ctypes.c_void_p(4096), None)
     assert st == 1
+
+
+@pytest.mark.parametrize("ldq,M,ldy,q,y", [(250, 4, 8, 4096, 8192), (256, 0, 8, 4096, 8192),
+                                          (256, 4, 3, 4096, 8192), (256, 4, 8, 4097, 8192),
+                                          (256, 4, 8, 4096, 0)])
+def test_gemm_rejects_bad_arguments(ldq, M, ldy, q, y):
+    lib = _lib()
+    m = _matrix()
+    st = lib.tern_gemm(ctypes.byref(m), ctypes.c_void_p(q), ldq, ctypes.c_void_p(4096), M,
+                       ctypes.c_void_p(y) if y else None, ldy, None)
+    assert st == 1, lib.tern_last_error()
+    assert b"tern_gemm" in lib.tern_last_error()

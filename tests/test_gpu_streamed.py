@@ -1,6 +1,6 @@
 """GPU parity of the streamed (persistent, evenly split) GEMV entry points:
-outputs match the oracle, repeated calls are identical, and the workspace is
-left zero (its counters reset) by every call."""
+outputs match the oracle, repeated calls are identical, and every call
+leaves the workspace all zero (it clears the partials it published)."""
 import numpy as np
 import pytest
 import torch
@@ -18,11 +18,9 @@ def tiled(fmt, w, sw):
     return make_matrix(fmt, w, sw).retile_scales()
 
 
-def counters(ws, N):
-    """The arrival counters, one per 32-row block, at the end of the workspace."""
-    rb = -(-N // 32)
-    flat = ws.view(torch.int32)
-    return flat[flat.numel() - rb:]
+def leftovers(ws):
+    """Nonzero words left in the workspace (must be none after a call)."""
+    return int(torch.count_nonzero(ws).item())
 
 
 @pytest.mark.parametrize("fmt", FMTS)
@@ -45,7 +43,7 @@ def test_streamed_gemv_matches_oracle(fmt, N, K, M, qflags):
         tern.tern_gemv_streamed(W, x[:, :K] if ldx == K else x, y, ws, qflags=qflags, M=M)
         outs.append(y.cpu().numpy())
     np.testing.assert_array_equal(outs[0], outs[1])
-    assert not counters(ws, N).any().item(), "the arrival counters must be left zero"
+    assert leftovers(ws) == 0, "the workspace must be left zero"
     q, s = oracle.act_quant(xh, fwht_block=128 if qflags & ROT else 0, rmsnorm=bool(qflags & RMS))
     ref = oracle.gemv(w, sw, q, s)
     assert np.max(np.abs(outs[0] - ref)) <= tolerance(ref)
@@ -66,7 +64,7 @@ def test_streamed_gateup(fmt, N, K, M):
     qo, so = oracle.act_quant(xh, fwht_block=128, rmsnorm=True)
     ref = oracle.gateup_swiglu(wg, sg, wu, su, qo, so)
     assert np.max(np.abs(h.cpu().numpy() - ref)) <= tolerance(ref)
-    assert not counters(ws, N).any().item()
+    assert leftovers(ws) == 0
 
 
 @pytest.mark.parametrize("fmt", FMTS)
@@ -124,4 +122,4 @@ def test_one_workspace_serves_calls_of_different_sizes(fmt):
             q, s = oracle.act_quant(xh, rmsnorm=True)
             ref = oracle.gemv(w, sw, q, s)
         assert np.max(np.abs(y.cpu().numpy() - ref)) <= tolerance(ref)
-    assert not counters(ws, 17408).any().item()
+    assert leftovers(ws) == 0

@@ -5,7 +5,7 @@ Some callers cannot call cudaMalloc: a plug-in whose host program owns all
 device memory through its own pool or budget, or code on a latency-critical
 path where cudaMalloc's implicit device-wide synchronisation would stall
 other streams.  For them the library keeps the streamed kernel's scratch
-(partial sums and arrival counters of the row blocks two CTAs share) in a
+(partial sums of the row blocks two CTAs share) in a
 fixed 1 MiB array of its own.  These tests check that this entry point gives
 the results of tern_gemv_streamed, which takes a caller workspace, on two
 calls in a row, and that it rejects sizes whose scratch would not fit.
