@@ -2,14 +2,16 @@
 """Benchmark of the ternary decode weight stream on B200.
 
 One step = one batch-1 decode step of a 64-layer 27B-shaped ternary layer
-stack (per layer: act quant, fused QKV GEMV, act quant, O GEMV + residual,
-act quant with 128-point Hadamard, fused gate/up + SwiGLU, act quant, down
-GEMV + residual), replayed as one CUDA graph.  The metric is the weight
-stream's algorithmic bytes (packed codes + fp16 group scales) per second,
-with the decode-step rate (tok/s-equivalent) beside it.
+stack, replayed as one CUDA graph.  Per layer four kernels (the streamed
+GEMV entry points, which quantise their fp32 input themselves): QKV GEMV,
+O GEMV + residual, fused gate/up + SwiGLU with the 128-point Hadamard
+rotation, down GEMV + residual.  The metric is the weight stream's
+algorithmic bytes (packed codes + fp16 group scales) per second, with the
+decode-step rate (tok/s-equivalent) beside it.  The line also carries the
+prefill GEMM (tern_gemm on the tensor cores) at M = 512 / 2048 / 8192.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--fmt base3|2bit] [--layers 64] [--M 1]
+                    [--fmt base3|2bit] [--layers 64] [--M 1] [--no-prefill]
 
 N > 1 runs N independent replicas (one process per GPU, launched by
 torch.distributed.run): the path has no cross-GPU exchange step.
@@ -48,6 +50,7 @@ def parse():
     ap.add_argument("--cpu-seconds", type=float, default=10.0,
                     help="target CPU time of the oracle baseline sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-prefill", action="store_true", help="skip the prefill GEMM measurement")
     return ap.parse_args()
 
 
@@ -59,6 +62,52 @@ def peaks():
         return float(p["hbm_gbs"]), "measured"
     except Exception:
         return FALLBACK_HBM_GBS, "fallback"
+
+
+def int8_peak():
+    """Dense int8 tensor peak: the measured bf16 burst figure x the nominal
+    int8 / bf16 ratio (4.5 / 2.25 PFLOP/s), else the recipe's fallback."""
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            return 2.0 * float(json.load(f)["bf16_tflops"]), "measured bf16 x 2"
+    except Exception:
+        return 2.0 * 1590.0, "fallback bf16 x 2"
+
+
+def prefill_gemm(fmt_id, Ms=(512, 2048, 8192), K=5120, N=17408, reps=10):
+    """tern_gemm on the gate/up shape (K = 5120, N = 17408) at prefill batch
+    sizes; TOPS = 2 M N K / device time (CUDA events, after warm-up).  W
+    (17.8 MB base-3) stays L2-resident across the token tiles, as in any
+    prefill; the kernel is tensor-core and epilogue bound, not HBM bound."""
+    import torch
+    from ternary_weight_decode_b200 import decode, tern
+    scratch = torch.empty(N * K, dtype=torch.int8, device="cuda")
+    W = decode.make_matrix(fmt_id, N, K, seed=977, stream=5, scratch=scratch)
+    del scratch
+    peak, kind = int8_peak()
+    gen = torch.Generator(device="cuda")
+    gen.manual_seed(1234)
+    res = []
+    for M in Ms:
+        q = torch.randint(-127, 128, (M, K), dtype=torch.int8, device="cuda", generator=gen)
+        s = torch.rand(M, device="cuda", generator=gen) * 0.01 + 0.001
+        y = torch.empty((M, N), dtype=torch.float32, device="cuda")
+        for _ in range(3):
+            tern.tern_gemm(W, q, s, y)
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(reps):
+            tern.tern_gemm(W, q, s, y)
+        e1.record()
+        e1.synchronize()
+        t = e0.elapsed_time(e1) / reps * 1e-3
+        tops = 2.0 * M * N * K / t / 1e12
+        res.append({"M": M, "ms": t * 1e3, "TOPS": tops, "frac": tops / peak})
+        del q, s, y
+    return {"workload": f"tern_gemm, K={K}, N={N}, int8 activations, fp16/128 group scales",
+            "unit": "TOPS", "peak": peak, "peak_kind": kind, "results": res}
 
 
 def dist_setup(n_gpus):
@@ -379,6 +428,11 @@ def main():
     cpu = None
     if world == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline(fmt_id, args.M, args.cpu_seconds)
+    prefill = None
+    if world == 1 and not args.no_prefill:
+        del graph
+        graph = None
+        prefill = prefill_gemm(fmt_id)
 
     line = {
         "metric": METRIC,
@@ -407,6 +461,7 @@ def main():
         "gpu_launches": model.launches_per_step() * args.steps,
         "clocks": clk,
         "cpu_baseline": cpu,
+        "prefill_gemm": prefill,
         "device_error": err,
         "output_finite": out_ok,
     }

@@ -208,7 +208,9 @@ tern_status tern_gemv(const tern_matrix *W, const int8_t *q, int32_t ldq,
  *  q: device int8 [M][ldq], 16-byte aligned, ldq >= K, ldq % 16 == 0
  *     (bytes past K are ignored).  s_x: device fp32 [M].
  *  y: device fp32 [M][ldy], ldy >= N; must not overlap q.
- * The caller owns every buffer; nothing is allocated.
+ * The caller owns every buffer; nothing is allocated.  While the device
+ * error word is set (a bounded wait in an earlier kernel ran out; see
+ * tern_device_error) the kernel returns without computing.
  */
 tern_status tern_gemm(const tern_matrix *W, const int8_t *q, int32_t ldq,
                       const float *s_x, int32_t M, float *y, int32_t ldy,

@@ -471,6 +471,23 @@ bool make_u8_tmap_2d(CUtensorMap *map, const void *base, uint64_t inner, uint64_
     return r == CUDA_SUCCESS;
 }
 
+bool make_weight_tmap3d(CUtensorMap *map, const void *packed, int N, int64_t row_stride,
+                        int sb_full, int box_sb) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn || sb_full < 1) return false;
+    // (byte in superblock, row, superblock): only whole superblocks, so no
+    // box reaches past a row's used bytes
+    cuuint64_t dims[3] = {static_cast<cuuint64_t>(kSBBytes), static_cast<cuuint64_t>(N),
+                          static_cast<cuuint64_t>(sb_full)};
+    cuuint64_t strides[2] = {static_cast<cuuint64_t>(row_stride), static_cast<cuuint64_t>(kSBBytes)};
+    cuuint32_t box[3] = {kSBBytes, 32, static_cast<cuuint32_t>(box_sb)};
+    cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void *>(packed), dims, strides,
+                    box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
 bool make_weight_tmap(CUtensorMap *map, const void *packed, int64_t row_bytes, int N,
                       int64_t row_stride) {
     return make_u8_tmap_2d(map, packed, static_cast<uint64_t>(row_bytes), static_cast<uint64_t>(N),

@@ -44,10 +44,16 @@ namespace {
 constexpr int kSkConsumers = 8;
 constexpr int kSkThreads = 32 * (kSkConsumers + 1);
 constexpr int kSkBar = 1;   // named barrier of the consumer warps
-constexpr int kSkKeep = 5;  // input blocks a consumer warp keeps in registers
+// Input blocks a consumer warp keeps in registers between the two passes
+// (one token row: K up to 9 x 8 warps x 2 CTAs x 128 = 18432 without reloads).
+template <int MT>
+__host__ __device__ constexpr int sk_keep() {
+    return MT == 1 ? 9 : 5;
+}
 constexpr int kSkMaxCluster = 4;
 constexpr int kSkSmemBudget = 112 * 1024;  // two CTAs per SM (programmatic launch overlap)
-constexpr int kSkMinRing = 8, kSkMaxRing = 24;
+constexpr int kSkMinRing = 8, kSkMaxRing = 24;  // unit slots, multiples of kSkChunk
+constexpr int kSkChunk = 4;                      // unit slots filled by one chunk of loads
 
 template <int FMT>
 __host__ __device__ constexpr int scb() {
@@ -55,7 +61,7 @@ __host__ __device__ constexpr int scb() {
 }
 
 struct SkParams {
-    int N, K, SB, RB, R;
+    int N, K, SB, SBF, RB, R;  // SBF: whole superblocks per row
     long long U;
     int nCTA, M, prefetch_ok, qflags;
     const uint16_t *tsc0;
@@ -218,6 +224,18 @@ __device__ __forceinline__ float amax4(const float (&r)[4]) {
     return fmaxf(fmaxf(fabsf(r[0]), fabsf(r[1])), fmaxf(fabsf(r[2]), fabsf(r[3])));
 }
 
+// Ring order of the items: chunk k holds units kCH .. kCH+CH-1 of matrix 0,
+// then the same units of matrix 1.  Item (unit ul of the range, matrix).
+template <int CH>
+__host__ __device__ __forceinline__ int sk_item_index(int ul, int mat) {
+    return (ul / CH) * kSkChunk + mat * CH + ul % CH;
+}
+template <int NMAT>
+__host__ __device__ inline int sk_items_max(long long U, int nCTA) {
+    const int units = static_cast<int>((U + nCTA - 1) / nCTA);
+    return (units + kSkChunk / NMAT - 1) / (kSkChunk / NMAT) * kSkChunk;
+}
+
 // Index of the tagged partial of (row block, matrix, token, lane).
 template <int NMAT, int MT>
 __device__ __forceinline__ int64_t tag_index(int rb, int mat, int m, int lane) {
@@ -227,8 +245,12 @@ __device__ __forceinline__ int64_t tag_index(int rb, int mat, int m, int lane) {
 template <int FMT, int MT, int MODE>
 __global__ void __launch_bounds__(kSkThreads, 2)
     gemv_stream_kernel(const __grid_constant__ CUtensorMap tm0,
-                       const __grid_constant__ CUtensorMap tm1, const SkParams p) {
+                       const __grid_constant__ CUtensorMap tm1,
+                       const __grid_constant__ CUtensorMap tm3_0,
+                       const __grid_constant__ CUtensorMap tm3_1, const SkParams p) {
     constexpr int NMAT = (MODE == kModeSwiglu) ? 2 : 1;
+    constexpr int CH = kSkChunk / NMAT;  // units of one matrix per ring chunk
+    constexpr int KEEP = sk_keep<MT>();
     constexpr int POS = Fmt<FMT>::kPos;
     constexpr int GPS = Fmt<FMT>::kGroups;
     constexpr int SCB = scb<FMT>();
@@ -239,9 +261,10 @@ __global__ void __launch_bounds__(kSkThreads, 2)
     const long long U = p.U;
     const int c = blockIdx.x;
     const long long u0 = U * c / p.nCTA, u1 = U * (c + 1) / p.nCTA;
-    const int nitems = static_cast<int>(u1 - u0) * NMAT;
-    const int items_max = static_cast<int>((U + p.nCTA - 1) / p.nCTA) * NMAT;
+    const int nunits = static_cast<int>(u1 - u0);
+    const int items_max = sk_items_max<NMAT>(U, p.nCTA);
     const SkLayout L = sk_layout<FMT, MT>(p.SB, items_max, R);
+    const int RC = R / kSkChunk;  // chunks in the ring
     uint8_t *ring_w = smem;
     uint8_t *ring_s = smem + L.ring_s_off;
     uint8_t *act = smem + L.act_off;
@@ -251,9 +274,9 @@ __global__ void __launch_bounds__(kSkThreads, 2)
     float *red = reinterpret_cast<float *>(smem + L.red_off);
     int *first_cnt = reinterpret_cast<int *>(smem + L.misc_off);
     float *slots = reinterpret_cast<float *>(smem + L.slots_off);
-    uint64_t *full = reinterpret_cast<uint64_t *>(smem + L.bar_off);
-    uint64_t *empty = full + R;
-    uint64_t *qbar1 = empty + R;  // the peers' partials of the row scale arrived
+    uint64_t *full = reinterpret_cast<uint64_t *>(smem + L.bar_off);  // per chunk
+    uint64_t *empty = full + RC;
+    uint64_t *qbar1 = empty + RC;  // the peers' partials of the row scale arrived
     uint64_t *qbar2 = qbar1 + 1;  // the peers' int8 input and group sums arrived
 
     const int C = static_cast<int>(cluster_nctarank());
@@ -264,10 +287,14 @@ __global__ void __launch_bounds__(kSkThreads, 2)
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     if (tid == 0) {
         prefetch_tmap(&tm0);
-        if (NMAT == 2) prefetch_tmap(&tm1);
-        for (int i = 0; i < R; ++i) {
+        prefetch_tmap(&tm3_0);
+        if (NMAT == 2) {
+            prefetch_tmap(&tm1);
+            prefetch_tmap(&tm3_1);
+        }
+        for (int i = 0; i < RC; ++i) {
             mbar_init(&full[i], 1);
-            mbar_init(&empty[i], 1);
+            mbar_init(&empty[i], kSkChunk);
         }
         *first_cnt = 0;
         mbar_init(qbar1, 1);
@@ -287,35 +314,54 @@ __global__ void __launch_bounds__(kSkThreads, 2)
         cluster_arrive();  // sends nothing: the exit barrier's arrival
         if (!p.prefetch_ok) pdl_wait();
         const uint64_t policy = l2_policy_evict_first();
+        // A chunk is CH consecutive units of each matrix: one 3-D box of CH
+        // whole superblocks when they lie in one row block (one TMA
+        // instruction per 16 KB: the tile issue rate, not HBM, bounds small
+        // boxes), else one 2-D box per unit; their scales in one bulk copy.
         // Positions advance incrementally: no division inside the loop.
-        int slot = 0, round = 0, mat = 0;
+        const int nchunks = (nunits + CH - 1) / CH;
+        int cs = 0, round = 0;
         int rb = static_cast<int>(u0 / p.SB), sb = static_cast<int>(u0 % p.SB);
         const uint8_t *sc_unit[2] = {reinterpret_cast<const uint8_t *>(p.tsc0) + u0 * SCB,
                                      reinterpret_cast<const uint8_t *>(p.tsc1) + u0 * SCB};
-        for (int j = 0; j < nitems; ++j) {
+        for (int k = 0; k < nchunks; ++k) {
             if (round > 0 &&
-                !__all_sync(0xffffffffu, mbar_wait_bounded(&empty[slot], (round - 1) & 1)))
+                !__all_sync(0xffffffffu, mbar_wait_bounded(&empty[cs], (round - 1) & 1)))
                 break;
+            const int nu = min(CH, nunits - k * CH);
             if (lane == 0) {
-                mbar_arrive_expect_tx(&full[slot], kTile + SCB);
-                tma_load_2d(ring_w + slot * kTile, mat ? &tm1 : &tm0, sb * kSBBytes, rb * 32,
-                            &full[slot], policy);
-                bulk_copy_g2s(ring_s + slot * SCB, sc_unit[mat], SCB, &full[slot], policy);
-            }
-            __syncwarp();
-            if (NMAT == 2 && mat == 0) {
-                mat = 1;
-            } else {
-                mat = 0;
-                sc_unit[0] += SCB;
-                sc_unit[1] += SCB;
-                if (++sb == p.SB) {
-                    sb = 0;
-                    ++rb;
+                mbar_arrive_expect_tx(&full[cs], nu * NMAT * (kTile + SCB));
+                const bool whole = nu == CH && sb + CH <= p.SBF;
+#pragma unroll
+                for (int mat = 0; mat < NMAT; ++mat) {
+                    const int slot0 = cs * kSkChunk + mat * CH;
+                    if (whole) {
+                        tma_load_3d(ring_w + slot0 * kTile, mat ? &tm3_1 : &tm3_0, 0, rb * 32, sb,
+                                    &full[cs], policy);
+                    } else {
+                        int r2 = rb, s2 = sb;
+                        for (int i = 0; i < nu; ++i) {
+                            tma_load_2d(ring_w + (slot0 + i) * kTile, mat ? &tm1 : &tm0,
+                                        s2 * kSBBytes, r2 * 32, &full[cs], policy);
+                            if (++s2 == p.SB) {
+                                s2 = 0;
+                                ++r2;
+                            }
+                        }
+                    }
+                    bulk_copy_g2s(ring_s + slot0 * SCB, sc_unit[mat], nu * SCB, &full[cs], policy);
                 }
             }
-            if (++slot == R) {
-                slot = 0;
+            __syncwarp();
+            sc_unit[0] += CH * SCB;
+            sc_unit[1] += CH * SCB;
+            sb += CH;
+            while (sb >= p.SB) {
+                sb -= p.SB;
+                ++rb;
+            }
+            if (++cs == RC) {
+                cs = 0;
                 ++round;
             }
         }
@@ -328,7 +374,6 @@ __global__ void __launch_bounds__(kSkThreads, 2)
         // row block is finished here (its start is here).
         const bool publish = static_cast<long long>(rb_lo) * p.SB < u0;
         const bool combine = static_cast<long long>(rb_hi + 1) * p.SB > u1;
-        const int n_first = publish ? static_cast<int>((static_cast<long long>(rb_lo + 1) * p.SB - u0) * NMAT) : 0;
         pdl_wait();
         // Residual of the first row block this warp finishes, fetched early.
         float res0[MT];
@@ -342,16 +387,16 @@ __global__ void __launch_bounds__(kSkThreads, 2)
         const bool rotate = (p.qflags & TERN_QUANT_FWHT128) != 0;
         const bool rms = (p.qflags & TERN_QUANT_RMSNORM) != 0;
 
-        // pass 1: loads first (kSkKeep blocks per warp in flight), then the
+        // pass 1: loads first (KEEP blocks per warp in flight), then the
         // rotation, max |.| and sum x^2 of this CTA's blocks
-        float v[MT][kSkKeep][4];
+        float v[MT][KEEP][4];
         float amax[MT], ss[MT];
 #pragma unroll
         for (int m = 0; m < MT; ++m) {
             amax[m] = 0.0f;
             ss[m] = 0.0f;
 #pragma unroll
-            for (int j = 0; j < kSkKeep; ++j) {
+            for (int j = 0; j < KEEP; ++j) {
                 const int b = b_lo + cw + kSkConsumers * j;
                 if (b < b_hi) {
                     load_block(p, m, b, lane, v[m][j]);
@@ -363,13 +408,13 @@ __global__ void __launch_bounds__(kSkThreads, 2)
 #pragma unroll
         for (int m = 0; m < MT; ++m)
 #pragma unroll
-            for (int j = 0; j < kSkKeep; ++j) {
+            for (int j = 0; j < KEEP; ++j) {
                 if (b_lo + cw + kSkConsumers * j >= b_hi) continue;
                 ss[m] += sumsq4(v[m][j]);
                 if (rotate) fwht128_warp(v[m][j], lane);
                 amax[m] = fmaxf(amax[m], amax4(v[m][j]));
             }
-        for (int b = b_lo + cw + kSkConsumers * kSkKeep; b < b_hi; b += kSkConsumers) {
+        for (int b = b_lo + cw + kSkConsumers * KEEP; b < b_hi; b += kSkConsumers) {
 #pragma unroll
             for (int m = 0; m < MT; ++m) {
                 float r[4];
@@ -381,7 +426,8 @@ __global__ void __launch_bounds__(kSkThreads, 2)
         }
 #pragma unroll
         for (int m = 0; m < MT; ++m) {
-            const float a = warp_max(amax[m]);
+            // max of non-negative floats = max of their bit patterns
+            const float a = __uint_as_float(__reduce_max_sync(0xffffffffu, __float_as_uint(amax[m])));
             const float s = warp_sum(ss[m]);
             if (lane == 0) {
                 red[(cw * MT + m) * 2 + 0] = a;
@@ -389,33 +435,49 @@ __global__ void __launch_bounds__(kSkThreads, 2)
             }
         }
         warpgroup_sync_n(kSkBar, kSkConsumers * 32);
-        if (ctid < MT) {
-            // this CTA's share (fixed warp order): kept here, sent to the peers
-            const int m = ctid;
+        // This CTA's share, combined by every thread in the same warp order.
+        float amax_c[MT], ss_c[MT];
+#pragma unroll
+        for (int m = 0; m < MT; ++m) {
             float a = 0.0f, s = 0.0f;
             for (int w = 0; w < kSkConsumers; ++w) {
                 a = fmaxf(a, red[(w * MT + m) * 2 + 0]);
                 s += red[(w * MT + m) * 2 + 1];
             }
-            xred[(rank * MT + m) * 2 + 0] = a;
-            xred[(rank * MT + m) * 2 + 1] = s;
-            for (int q = 0; q < C; ++q)
-                if (q != rank)
-                    st_async_v2f32(map_shared_rank(xred + (rank * MT + m) * 2, q), a, s,
-                                   map_shared_rank(qbar1, q));
+            amax_c[m] = a;
+            ss_c[m] = s;
         }
-        warpgroup_sync_n(kSkBar, kSkConsumers * 32);
-        const bool ok1 = mbar_wait_cluster_bounded(qbar1, 0);
-        // Row scale from the cluster's shares (same order in every CTA).
+        bool ok1 = true;
+        if (C > 1) {
+            // shares of the cluster: sent to the peers, combined in rank order
+            if (ctid < MT) {
+                const int m = ctid;
+                xred[(rank * MT + m) * 2 + 0] = amax_c[m];
+                xred[(rank * MT + m) * 2 + 1] = ss_c[m];
+                for (int q = 0; q < C; ++q)
+                    if (q != rank)
+                        st_async_v2f32(map_shared_rank(xred + (rank * MT + m) * 2, q), amax_c[m],
+                                       ss_c[m], map_shared_rank(qbar1, q));
+            }
+            warpgroup_sync_n(kSkBar, kSkConsumers * 32);
+            ok1 = mbar_wait_cluster_bounded(qbar1, 0);
+#pragma unroll
+            for (int m = 0; m < MT; ++m) {
+                float a = 0.0f, s = 0.0f;
+                for (int q = 0; q < C; ++q) {
+                    const bool have = ok1 || q == rank;
+                    a = fmaxf(a, have ? xred[(q * MT + m) * 2 + 0] : 0.0f);
+                    s += have ? xred[(q * MT + m) * 2 + 1] : 0.0f;
+                }
+                amax_c[m] = a;
+                ss_c[m] = s;
+            }
+        }
+        // Row scale (the same in every CTA).
         float inv[MT];
 #pragma unroll
         for (int m = 0; m < MT; ++m) {
-            float a = 0.0f, s = 0.0f;
-            for (int q = 0; q < C; ++q) {
-                const bool have = ok1 || q == rank;
-                a = fmaxf(a, have ? xred[(q * MT + m) * 2 + 0] : 0.0f);
-                s += have ? xred[(q * MT + m) * 2 + 1] : 0.0f;
-            }
+            const float a = amax_c[m], s = ss_c[m];
             float iv = 0.0f, sc = 0.0f;
             if (a > 0.0f) {
                 iv = __fdiv_rn(127.0f, a);
@@ -442,18 +504,18 @@ __global__ void __launch_bounds__(kSkThreads, 2)
                 qsum += qi;
                 packed |= (static_cast<uint32_t>(qi) & 0xffu) << (8 * e);
             }
-            qsum = warp_sum_int(qsum);
+            qsum = __reduce_add_sync(0xffffffffu, qsum);  // one warp-wide reduction
             *reinterpret_cast<uint32_t *>(act + m * L.Kpad + 128 * b + 4 * lane) = packed;
             if (lane == 0) sq[(m * L.GT + b) * 4] = qsum;
         };
 #pragma unroll
         for (int m = 0; m < MT; ++m)
 #pragma unroll
-            for (int j = 0; j < kSkKeep; ++j) {
+            for (int j = 0; j < KEEP; ++j) {
                 const int b = b_lo + cw + kSkConsumers * j;
                 if (b < b_hi) quant_block(m, b, v[m][j]);
             }
-        for (int b = b_lo + cw + kSkConsumers * kSkKeep; b < b_hi; b += kSkConsumers) {
+        for (int b = b_lo + cw + kSkConsumers * KEEP; b < b_hi; b += kSkConsumers) {
 #pragma unroll
             for (int m = 0; m < MT; ++m) {
                 float r[4];
@@ -481,14 +543,22 @@ __global__ void __launch_bounds__(kSkThreads, 2)
         // on it (and the peers' copies out of their shared memory are done).
         cluster_arrive();
 
-        // items, round-robin over the consumer warps; the slot is handed back
-        // as soon as the item sits in registers.  Slot, phase and superblock
-        // advance incrementally (R >= kSkConsumers: at most one wrap a step).
-        int slot = cw, phase = 0;
-        int sb = static_cast<int>((u0 + cw / NMAT) % p.SB);
-        for (int j = cw; j < nitems; j += kSkConsumers) {
+        // items, round-robin over the consumer warps (a warp always takes the
+        // same position in a chunk, hence the same matrix); the item is copied
+        // to registers and its chunk slot handed back at once.  Chunk, phase
+        // and superblock advance incrementally (two chunks a step).
+        const int pos = cw % kSkChunk, mat_w = pos / CH, uoff = pos % CH;
+        int kc = cw / kSkChunk;
+        int kcs = kc % RC, phase = (kc / RC) & 1;
+        int sb = static_cast<int>((u0 + kc * CH + uoff) % p.SB);
+        const int n_first = publish ? static_cast<int>(static_cast<long long>(rb_lo + 1) * p.SB - u0) : 0;
+        for (;; kc += kSkConsumers / kSkChunk) {
+            const int ul = kc * CH + uoff;
+            if (ul >= nunits) break;
+            const int j = kc * kSkChunk + pos;
             const bool ok =
-                ok2 && __all_sync(0xffffffffu, mbar_wait_bounded(&full[slot], phase));
+                ok2 && __all_sync(0xffffffffu, mbar_wait_bounded(&full[kcs], phase));
+            const int slot = kcs * kSkChunk + pos;
             float yacc[MT];
             if (ok) {
                 uint32_t words[32];
@@ -508,24 +578,24 @@ __global__ void __launch_bounds__(kSkThreads, 2)
 #pragma unroll
                 for (int g = 0; g < GPS; ++g) sc[g] = __half2float(__ushort_as_half(st[g]));
                 __syncwarp();
-                if (lane == 0) mbar_arrive(&empty[slot]);
+                if (lane == 0) mbar_arrive(&empty[kcs]);
                 sk_item<FMT, MT>(words, sc, act + sb * POS, L.Kpad, sq + sb * GPS * 4, L.GT, yacc);
             } else {
                 __syncwarp();
-                if (lane == 0) mbar_arrive(&empty[slot]);
+                if (lane == 0) mbar_arrive(&empty[kcs]);
 #pragma unroll
                 for (int m = 0; m < MT; ++m) yacc[m] = 0.0f;
             }
 #pragma unroll
             for (int m = 0; m < MT; ++m) slots[(j * MT + m) * 32 + lane] = yacc[m];
-            slot += kSkConsumers;
-            if (slot >= R) {
-                slot -= R;
+            kcs += kSkConsumers / kSkChunk;
+            if (kcs >= RC) {
+                kcs -= RC;
                 phase ^= 1;
             }
-            sb += kSkConsumers / NMAT;
+            sb += (kSkConsumers / kSkChunk) * CH;
             while (sb >= p.SB) sb -= p.SB;
-            if (j < n_first) {
+            if (ul < n_first) {
                 // The last warp to finish an item of the cut first row block
                 // publishes that row block's partial (value and tag in one
                 // 64-bit store) for the CTA holding its start.
@@ -536,16 +606,15 @@ __global__ void __launch_bounds__(kSkThreads, 2)
                     done = atomicAdd(first_cnt, 1);
                 }
                 done = __shfl_sync(0xffffffffu, done, 0);
-                if (done == n_first - 1) {
+                if (done == n_first * NMAT - 1) {
                     __threadfence_block();
-                    const long long ue = static_cast<long long>(rb_lo + 1) * p.SB;
 #pragma unroll
                     for (int mat = 0; mat < NMAT; ++mat)
 #pragma unroll
                         for (int m = 0; m < MT; ++m) {
                             float s = 0.0f;
-                            for (long long uu = u0; uu < ue; ++uu)
-                                s += slots[(((uu - u0) * NMAT + mat) * MT + m) * 32 + lane];
+                            for (int uu = 0; uu < n_first; ++uu)
+                                s += slots[(sk_item_index<CH>(uu, mat) * MT + m) * 32 + lane];
                             st_relaxed_gpu_u64(p.ws_tag + tag_index<NMAT, MT>(rb_lo, mat, m, lane),
                                                (1ull << 32) | __float_as_uint(s));
                         }
@@ -567,7 +636,7 @@ __global__ void __launch_bounds__(kSkThreads, 2)
                 for (int m = 0; m < MT; ++m) {
                     float s = 0.0f;
                     for (long long u = ua; u < ub; ++u)
-                        s += slots[(((u - u0) * NMAT + mat) * MT + m) * 32 + lane];
+                        s += slots[(sk_item_index<CH>(static_cast<int>(u - u0), mat) * MT + m) * 32 + lane];
                     tot[mat][m] = s;
                 }
             if (rb == rb_hi && combine) {
@@ -658,6 +727,7 @@ cudaError_t launch_sk(const StreamLaunch &S, cudaStream_t s, const char **why) {
     p.N = S.N;
     p.K = S.K;
     p.SB = static_cast<int>(ceil_div(S.row_bytes, kSBBytes));
+    p.SBF = static_cast<int>(S.row_bytes / kSBBytes);
     p.RB = static_cast<int>(ceil_div(S.N, 32));
     p.U = static_cast<long long>(p.RB) * p.SB;
     p.M = S.M;
@@ -682,28 +752,44 @@ cudaError_t launch_sk(const StreamLaunch &S, cudaStream_t s, const char **why) {
         if (e != cudaSuccess) return e;
         plan_c[dev] = choose_cluster(kern, S.num_sms, &plan_n[dev]);
     }
+    // The smallest cluster whose CTAs hold their share of the input blocks in
+    // registers (no reloads); a single CTA needs no exchange at all.
+    const int GT = p.SB * Fmt<FMT>::kGroups;
+    int C = 1;
+    while (C < plan_c[dev] && ceil_div(ceil_div(GT, C), kSkConsumers) > sk_keep<MT>()) C *= 2;
     // every range holds >= SB units, so a row block meets at most 2 ranges
     long long want = p.U / p.SB;
-    if (want > plan_n[dev]) want = plan_n[dev];
+    if (want > (C > 1 ? plan_n[dev] : S.num_sms)) want = C > 1 ? plan_n[dev] : S.num_sms;
     if (want < 1) want = 1;
-    int C = plan_c[dev];
     while (C > 1 && want < C) C /= 2;
     p.nCTA = static_cast<int>((want / C) * C);
-    const int items_max = static_cast<int>((p.U + p.nCTA - 1) / p.nCTA) * NMAT;
-    // ring depth: as many slots as fit the two-CTAs-per-SM budget
+    const int items_max = sk_items_max<NMAT>(p.U, p.nCTA);
+    // ring depth: as many whole chunks as fit the two-CTAs-per-SM budget
     int R = kSkMaxRing;
-    while (R > kSkMinRing && sk_layout<FMT, MT>(p.SB, items_max, R).total > kSkSmemBudget) --R;
+    while (R > kSkMinRing && sk_layout<FMT, MT>(p.SB, items_max, R).total > kSkSmemBudget)
+        R -= kSkChunk;
     p.R = R;
     const SkLayout L = sk_layout<FMT, MT>(p.SB, items_max, R);
     if (L.total > 227 * 1024) {
         *why = "shared memory plan of the streamed kernel exceeds 227 KB";
         return cudaErrorInvalidValue;
     }
-    CUtensorMap tm0, tm1;
+    CUtensorMap tm0, tm1, tm3_0, tm3_1;
+    constexpr int CH = kSkChunk / NMAT;
     if (!make_weight_tmap(&tm0, S.packed[0], S.row_bytes, S.N, S.row_stride) ||
         !make_weight_tmap(&tm1, S.packed[NMAT - 1], S.row_bytes, S.N, S.row_stride)) {
         *why = "cuTensorMapEncodeTiled failed or is unavailable";
         return cudaErrorInvalidValue;
+    }
+    if (p.SBF >= 1) {
+        if (!make_weight_tmap3d(&tm3_0, S.packed[0], S.N, S.row_stride, p.SBF, CH) ||
+            !make_weight_tmap3d(&tm3_1, S.packed[NMAT - 1], S.N, S.row_stride, p.SBF, CH)) {
+            *why = "cuTensorMapEncodeTiled (3-D) failed";
+            return cudaErrorInvalidValue;
+        }
+    } else {
+        tm3_0 = tm0;  // never used: no whole superblock, every chunk takes 2-D boxes
+        tm3_1 = tm1;
     }
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(p.nCTA, 1, 1);
@@ -719,7 +805,7 @@ cudaError_t launch_sk(const StreamLaunch &S, cudaStream_t s, const char **why) {
     attr[1].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = C > 1 ? 2 : 1;
-    e = cudaLaunchKernelEx(&cfg, kern, tm0, tm1, p);
+    e = cudaLaunchKernelEx(&cfg, kern, tm0, tm1, tm3_0, tm3_1, p);
     if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }

@@ -103,6 +103,10 @@ cudaError_t launch_act_stats(const float *x, int M, int K, int ldx, float *stats
                              cudaStream_t s);
 cudaError_t read_clear_device_error(int *value, cudaStream_t s);
 
+// 3-D view (byte in superblock, row, superblock) of a packed matrix's whole
+// superblocks: one box = box_sb consecutive superblocks of 32 rows.
+bool make_weight_tmap3d(CUtensorMap *map, const void *packed, int N, int64_t row_stride,
+                        int sb_full, int box_sb);
 // 2-D uint8 tensor map with 128-byte swizzle (tern_gemv.cu).
 bool make_u8_tmap_2d(CUtensorMap *map, const void *base, uint64_t inner, uint64_t rows,
                      uint64_t stride, uint32_t box_inner, uint32_t box_rows);
