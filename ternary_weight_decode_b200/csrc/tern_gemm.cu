@@ -12,18 +12,20 @@
 //  * warp 0 (TMA): per 128-byte superblock of codes, the 128 x 128 B code
 //    tile; per group of 128 K, the 128 x 128 B activation tile -- both with
 //    128-byte swizzle, no multicast;
-//  * warps 2..5 (decode, one weight row per thread): the row's 32 code words
-//    of the superblock into registers, then per group the signed int8
-//    weights w = t - 1 into a 128 x 128 B tile in the 128-byte-swizzled
-//    K-major layout the MMA reads (trits never leave the SM);
+//  * warps 2..9 (decode; a thread = one weight row, one 64-K half of each
+//    group): the row's 32 code words of the superblock into registers, then
+//    per group the signed int8 weights w = t - 1 into a 128 x 128 B tile in
+//    the 128-byte-swizzled K-major layout the MMA reads (trits never leave
+//    the SM);
 //  * warp 1 (MMA, one thread): per group four tcgen05.mma (K = 32 each), A =
-//    weights, B = activations, int32 accumulator in tensor memory -- two
-//    accumulator buffers of 128 columns, so group g+1 is multiplied while
-//    group g is drained;
-//  * warps 6..13 (epilogue, two per tensor-memory lane quarter, 64 token
-//    columns each): per group tcgen05.ld of the int32 partials, exact int ->
-//    float, acc += s_w[n][g] * P in fp32 registers (group order, as the
-//    definition reads); at the end Y = s_x[m] * acc.
+//    weights, B = activations, int32 accumulator in tensor memory -- four
+//    accumulator buffers of 128 columns (all 512), so the tensor cores run
+//    up to three groups ahead of the epilogue;
+//  * warps 10..17 (epilogue, two per tensor-memory lane quarter, 64 token
+//    columns each): the tile's group scales into shared memory once, then
+//    per group tcgen05.ld of the int32 partials, int -> float (exact: the
+//    partials are below 2^15), acc += s_w[n][g] * P in fp32 registers (group
+//    order, as the definition reads); at the end Y = s_x[m] * acc.
 // The per-group scale is why the accumulator is drained every 128 K: the
 // tensor cores accumulate only the exact integer partial of one group.
 #include "tern_gemv_common.cuh"
@@ -38,11 +40,14 @@ constexpr int kGmTile = 128 * 128;  // bytes of one 128 x 128 B int8 tile
 constexpr int kGmCodeStages = 2;
 constexpr int kGmActStages = 4;
 constexpr int kGmAStages = 2;
-constexpr int kGmDecodeWarps = 4;
+constexpr int kGmDecodeWarps = 8;
 constexpr int kGmEpiWarps = 8;
+constexpr int kGmEpiCols = kGmTileM * 4 / kGmEpiWarps;  // token columns per epilogue warp
 constexpr int kGmWarps = 2 + kGmDecodeWarps + kGmEpiWarps;
 constexpr int kGmThreads = 32 * kGmWarps;
-constexpr int kGmTmemCols = 256;  // two 128-column int32 accumulators
+constexpr int kGmAccBufs = 4;
+constexpr int kGmTmemCols = 128 * kGmAccBufs;  // four 128-column int32 accumulators
+constexpr int kGmEpiBar = 1;                   // named barrier of the epilogue warps
 
 struct GemmParams {
     int N, K, M, G, SB;
@@ -59,16 +64,52 @@ struct GemmSmem {
     uint64_t code_full[kGmCodeStages], code_empty[kGmCodeStages];
     uint64_t act_full[kGmActStages], act_empty[kGmActStages];
     uint64_t a_full[kGmAStages], a_empty[kGmAStages];
-    uint64_t acc_full[2], acc_empty[2];
+    uint64_t acc_full[kGmAccBufs], acc_empty[kGmAccBufs];
     uint32_t tmem_base;
+    // followed by the tile's group scales, fp16 [G][128] (group-major)
 };
 
 // w = t - 1 on four packed digits t in {0, 1, 2}: no byte carries.
 __device__ __forceinline__ uint32_t signed_trits(uint32_t t) { return (t + 0x7F7F7F7Fu) ^ 0x80808080u; }
 
-// Exact int -> float for |v| < 2^22 on the full-rate pipes.
-__device__ __forceinline__ float int_to_float_exact(uint32_t v) {
-    return __int_as_float(static_cast<int>(v) + 0x4B400000) - 12582912.0f;
+// One half (64 K) of group gg of a weight row: its 16 words of four signed
+// weights, stored as four 16-byte chunks of the swizzled A tile row.
+template <int FMT, int H>
+__device__ __forceinline__ void decode_half(const uint32_t (&words)[32], int gg, uint8_t *arow, int r) {
+    uint32_t wq[16];
+    if constexpr (FMT == TERN_FMT_BASE3) {
+        // D3: t-word d of the superblock (positions 4d..4d+3) is digit d % 5
+        // of code word d / 5
+        const int d0 = 32 * gg + 16 * H;
+#pragma unroll
+        for (int cw = d0 / 5; cw <= (d0 + 15) / 5; ++cw) {
+            uint32_t t[5];
+            decode_d3(words[cw], t);
+#pragma unroll
+            for (int i = 0; i < 5; ++i) {
+                const int d = 5 * cw + i - d0;
+                if (d >= 0 && d < 16) wq[d] = signed_trits(t[i]);
+            }
+        }
+    } else {
+        // D2: code word w holds positions 16w + 4i + j in bits [2i, 2i+1] of
+        // byte j; group gg = words 8gg .. 8gg+7
+#pragma unroll
+        for (int w4 = 0; w4 < 4; ++w4) {
+            const uint32_t X = words[8 * gg + 4 * H + w4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) wq[4 * w4 + i] = signed_trits((X >> (2 * i)) & 0x03030303u);
+        }
+    }
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+        uint4 v;
+        v.x = wq[4 * c + 0];
+        v.y = wq[4 * c + 1];
+        v.z = wq[4 * c + 2];
+        v.w = wq[4 * c + 3];
+        *reinterpret_cast<uint4 *>(arow + (((4 * H + c) ^ (r & 7)) << 4)) = v;
+    }
 }
 
 template <int FMT>
@@ -101,7 +142,7 @@ __global__ void __launch_bounds__(kGmThreads, 1)
             mbar_init(&S.a_full[i], kGmDecodeWarps);
             mbar_init(&S.a_empty[i], 1);
         }
-        for (int i = 0; i < 2; ++i) {
+        for (int i = 0; i < kGmAccBufs; ++i) {
             mbar_init(&S.acc_full[i], 1);
             mbar_init(&S.acc_empty[i], kGmEpiWarps);
         }
@@ -144,10 +185,11 @@ __global__ void __launch_bounds__(kGmThreads, 1)
         if (lane == 0) {
             const uint32_t idesc = idesc_i8(kGmTileN, kGmTileM, 1, 1);
             for (int g = 0; g < G; ++g) {
-                const int as = g % kGmAStages, qs = g % kGmActStages, buf = g & 1;
+                const int as = g % kGmAStages, qs = g % kGmActStages, buf = g % kGmAccBufs;
                 bool ok = mbar_wait_bounded(&S.a_full[as], (g / kGmAStages) & 1);
                 ok = ok && mbar_wait_bounded(&S.act_full[qs], (g / kGmActStages) & 1);
-                if (g >= 2) ok = ok && mbar_wait_bounded(&S.acc_empty[buf], ((g >> 1) - 1) & 1);
+                if (g >= kGmAccBufs)
+                    ok = ok && mbar_wait_bounded(&S.acc_empty[buf], ((g / kGmAccBufs) - 1) & 1);
                 if (!ok) break;
                 tc_fence_after_sync();
                 const uint32_t a0 = smem_u32(S.a[as]), b0 = smem_u32(S.act[qs]);
@@ -162,7 +204,9 @@ __global__ void __launch_bounds__(kGmThreads, 1)
         }
     } else if (warp < 2 + kGmDecodeWarps) {
         // ---------------------------------------------------------- decode
-        const int r = tid - 64;  // weight row of the tile, 0..127
+        const int dt = tid - 64;
+        const int r = dt & (kGmTileN - 1);  // weight row of the tile
+        const int half = dt >> 7;           // which 64 K of each group (warp-uniform)
         int g = 0;
         for (int sb = 0; sb < p.SB && g < G; ++sb) {
             const int cs = sb % kGmCodeStages;
@@ -190,41 +234,10 @@ __global__ void __launch_bounds__(kGmThreads, 1)
                                 mbar_wait_bounded(&S.a_empty[as], ((g / kGmAStages) - 1) & 1)))
                     break;
                 uint8_t *arow = S.a[as] + r * 128;
-                // 32 words of 4 signed weights = this row's 128 K of group g
-                uint32_t wq[32];
-                if constexpr (FMT == TERN_FMT_BASE3) {
-                    // D3: t-word d of the superblock (positions 4d..4d+3) is
-                    // digit d % 5 of code word d / 5
-#pragma unroll
-                    for (int cw = (32 * gg) / 5; cw <= (32 * gg + 31) / 5; ++cw) {
-                        uint32_t t[5];
-                        decode_d3(words[cw], t);
-#pragma unroll
-                        for (int i = 0; i < 5; ++i) {
-                            const int d = 5 * cw + i - 32 * gg;
-                            if (d >= 0 && d < 32) wq[d] = signed_trits(t[i]);
-                        }
-                    }
-                } else {
-                    // D2: code word w holds positions 16w + 4i + j in bits
-                    // [2i, 2i+1] of byte j; group gg = words 8gg .. 8gg+7
-#pragma unroll
-                    for (int w8 = 0; w8 < 8; ++w8) {
-                        const uint32_t X = words[8 * gg + w8];
-#pragma unroll
-                        for (int i = 0; i < 4; ++i)
-                            wq[4 * w8 + i] = signed_trits((X >> (2 * i)) & 0x03030303u);
-                    }
-                }
-#pragma unroll
-                for (int c = 0; c < 8; ++c) {
-                    uint4 v;
-                    v.x = wq[4 * c + 0];
-                    v.y = wq[4 * c + 1];
-                    v.z = wq[4 * c + 2];
-                    v.w = wq[4 * c + 3];
-                    *reinterpret_cast<uint4 *>(arow + ((c ^ (r & 7)) << 4)) = v;
-                }
+                if (half == 0)
+                    decode_half<FMT, 0>(words, gg, arow, r);
+                else
+                    decode_half<FMT, 1>(words, gg, arow, r);
                 fence_proxy_async_smem();  // read by the tensor cores
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&S.a_full[as]);
@@ -233,43 +246,49 @@ __global__ void __launch_bounds__(kGmThreads, 1)
         }
     } else {
         // -------------------------------------------------------- epilogue
-        const int e = warp - 2 - kGmDecodeWarps;  // 0..7
-        const int quarter = warp & 3;             // tensor-memory lanes it reaches
-        const int half = e >> 2;                  // token columns [64 half, 64 half + 64)
-        const int n = n0 + 32 * quarter + lane;
+        const int e = warp - 2 - kGmDecodeWarps;      // 0..7
+        const int quarter = warp & 3;                  // tensor-memory lanes it reaches
+        const int c0 = (e >> 2) * kGmEpiCols;         // its token columns
+        const int r = 32 * quarter + lane;             // tile row
+        const int n = n0 + r;
         const uint32_t lane_addr = static_cast<uint32_t>(32 * quarter) << 16;
-        float acc[64];
+        // the tile's scales, group-major (conflict-free reads below)
+        uint16_t *ssc = reinterpret_cast<uint16_t *>(&S + 1);
+        for (int idx = tid - 32 * (2 + kGmDecodeWarps); idx < kGmTileN * G; idx += 32 * kGmEpiWarps) {
+            const int rr = idx / G, gg = idx % G;
+            ssc[gg * kGmTileN + rr] = n0 + rr < p.N ? p.scales[static_cast<int64_t>(n0 + rr) * G + gg] : 0;
+        }
+        warpgroup_sync_n(kGmEpiBar, 32 * kGmEpiWarps);
+        float acc[kGmEpiCols];
 #pragma unroll
-        for (int c = 0; c < 64; ++c) acc[c] = 0.0f;
-        const uint16_t *srow = p.scales + static_cast<int64_t>(n < p.N ? n : 0) * G;
-        float s_next = n < p.N ? __half2float(__ushort_as_half(__ldg(srow))) : 0.0f;
+        for (int c = 0; c < kGmEpiCols; ++c) acc[c] = 0.0f;
         for (int g = 0; g < G; ++g) {
-            const int buf = g & 1;
-            const float s = s_next;
-            if (g + 1 < G && n < p.N) s_next = __half2float(__ushort_as_half(__ldg(srow + g + 1)));
-            const bool ok = __all_sync(0xffffffffu, mbar_wait_bounded(&S.acc_full[buf], (g >> 1) & 1));
+            const int buf = g % kGmAccBufs;
+            const float s = __half2float(__ushort_as_half(ssc[g * kGmTileN + r]));
+            const bool ok =
+                __all_sync(0xffffffffu, mbar_wait_bounded(&S.acc_full[buf], (g / kGmAccBufs) & 1));
             if (!ok) break;
             tc_fence_after_sync();
-            uint32_t v[32];
+            uint32_t v[16];
 #pragma unroll
-            for (int h = 0; h < 2; ++h) {
-                tmem_ld32(tmem + lane_addr + buf * 128 + 64 * half + 32 * h, v);
+            for (int h = 0; h < kGmEpiCols / 16; ++h) {
+                tmem_ld16(tmem + lane_addr + buf * 128 + c0 + 16 * h, v);
                 tmem_wait_ld();
-                if (h == 1) {
+                if (h == kGmEpiCols / 16 - 1) {
                     tc_fence_before_sync();
                     __syncwarp();
                     if (lane == 0) mbar_arrive(&S.acc_empty[buf]);
                 }
 #pragma unroll
-                for (int c = 0; c < 32; ++c)
-                    acc[32 * h + c] = fmaf(s, int_to_float_exact(v[c]), acc[32 * h + c]);
+                for (int c = 0; c < 16; ++c)
+                    acc[16 * h + c] = fmaf(s, __int2float_rn(static_cast<int>(v[c])), acc[16 * h + c]);
             }
         }
         pdl_wait();  // s_x comes from the previous kernel
         if (n < p.N) {
 #pragma unroll
-            for (int c = 0; c < 64; ++c) {
-                const int m = m0 + 64 * half + c;
+            for (int c = 0; c < kGmEpiCols; ++c) {
+                const int m = m0 + c0 + c;
                 if (m < p.M) p.y[static_cast<int64_t>(m) * p.ldy + n] = __ldg(p.s_x + m) * acc[c];
             }
         }
@@ -287,7 +306,7 @@ bool make_tmap_2d(CUtensorMap *map, const void *base, uint64_t inner, uint64_t r
     return make_u8_tmap_2d(map, base, inner, rows, stride, 128, box_rows);
 }
 
-size_t gemm_smem_bytes() { return sizeof(GemmSmem) + 1024; }
+size_t gemm_smem_bytes(int G) { return sizeof(GemmSmem) + static_cast<size_t>(G) * kGmTileN * 2 + 1024; }
 
 }  // namespace
 
@@ -310,7 +329,11 @@ cudaError_t launch_gemm(const GemmLaunch &L, cudaStream_t s, const char **why) {
         *why = "cuTensorMapEncodeTiled failed or is unavailable";
         return cudaErrorInvalidValue;
     }
-    const size_t smem = gemm_smem_bytes();
+    const size_t smem = gemm_smem_bytes(p.G);
+    if (smem > 227 * 1024) {
+        *why = "K too large for the shared-memory scale block of the prefill GEMM (K <= 40960)";
+        return cudaErrorInvalidValue;
+    }
     cudaError_t e;
     auto kern = L.fmt == TERN_FMT_BASE3 ? gemm_kernel<TERN_FMT_BASE3> : gemm_kernel<TERN_FMT_2BIT>;
     e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
