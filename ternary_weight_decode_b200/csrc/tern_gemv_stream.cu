@@ -200,6 +200,18 @@ __device__ __forceinline__ void sk_item(const uint32_t (&words)[32],
     }
 }
 
+// Four floats at p (16-byte aligned) when `pred`, else zeros; one
+// predicated L2 load, never reordered against the other volatile loads.
+__device__ __forceinline__ void ld_cg_f32x4_pred(const float *p, bool pred, float (&r)[4]) {
+    asm volatile(
+        "{\n\t.reg .pred q;\n\t"
+        "setp.ne.b32 q, %5, 0;\n\t"
+        "mov.b32 %0, 0;\n\tmov.b32 %1, 0;\n\tmov.b32 %2, 0;\n\tmov.b32 %3, 0;\n\t"
+        "@q ld.global.cg.v4.f32 {%0, %1, %2, %3}, [%4];\n\t}"
+        : "=f"(r[0]), "=f"(r[1]), "=f"(r[2]), "=f"(r[3])
+        : "l"(p), "r"(static_cast<int>(pred)));
+}
+
 // Lane's 4 values of 128-block b of token row m (zero past K and for m >= M).
 __device__ __forceinline__ void load_block(const SkParams &p, int m, int b, int lane, float (&r)[4]) {
     r[0] = r[1] = r[2] = r[3] = 0.0f;
@@ -391,6 +403,9 @@ __global__ void __launch_bounds__(kSkThreads, 2)
         // rotation, max |.| and sum x^2 of this CTA's blocks
         float v[MT][KEEP][4];
         float amax[MT], ss[MT];
+        // Every full 4-value load is issued before any is used (predicated
+        // volatile loads: the compiler may not interleave them with their
+        // uses); a block ending past K is read by load_block afterwards.
 #pragma unroll
         for (int m = 0; m < MT; ++m) {
             amax[m] = 0.0f;
@@ -398,13 +413,19 @@ __global__ void __launch_bounds__(kSkThreads, 2)
 #pragma unroll
             for (int j = 0; j < KEEP; ++j) {
                 const int b = b_lo + cw + kSkConsumers * j;
-                if (b < b_hi) {
-                    load_block(p, m, b, lane, v[m][j]);
-                } else {
-                    v[m][j][0] = v[m][j][1] = v[m][j][2] = v[m][j][3] = 0.0f;
-                }
+                const int k = 128 * b + 4 * lane;
+                const bool full = b < b_hi && m < p.M && k + 4 <= p.K;
+                ld_cg_f32x4_pred(p.x + static_cast<int64_t>(m) * p.ldx + k, full, v[m][j]);
             }
         }
+#pragma unroll
+        for (int m = 0; m < MT; ++m)
+#pragma unroll
+            for (int j = 0; j < KEEP; ++j) {
+                const int b = b_lo + cw + kSkConsumers * j;
+                const int k = 128 * b + 4 * lane;
+                if (b < b_hi && m < p.M && k < p.K && k + 4 > p.K) load_block(p, m, b, lane, v[m][j]);
+            }
 #pragma unroll
         for (int m = 0; m < MT; ++m)
 #pragma unroll
@@ -479,12 +500,14 @@ __global__ void __launch_bounds__(kSkThreads, 2)
         for (int m = 0; m < MT; ++m) {
             const float a = amax_c[m], s = ss_c[m];
             float iv = 0.0f, sc = 0.0f;
+            // inv decides every int8 code: IEEE division, as the oracle.  The
+            // output scale only multiplies fp32 results: approximate forms.
             if (a > 0.0f) {
                 iv = __fdiv_rn(127.0f, a);
-                sc = __fdiv_rn(a, 127.0f);
-                if (rotate) sc = __fmul_rn(sc, kInvSqrt128);
+                sc = a * (1.0f / 127.0f);
+                if (rotate) sc *= kInvSqrt128;
             }
-            if (rms) sc = sc / sqrtf(s / static_cast<float>(p.K) + 1e-6f);
+            if (rms) sc *= rsqrtf(s / static_cast<float>(p.K) + 1e-6f);
             inv[m] = iv;
             if (ctid == 0) sx[m] = sc;
         }
@@ -492,19 +515,17 @@ __global__ void __launch_bounds__(kSkThreads, 2)
         // pass 2: int8 codes and group sums of this CTA's blocks, written
         // here, then one bulk copy of the share to each peer
         auto quant_block = [&](int m, int b, const float (&r)[4]) {
-            uint32_t packed = 0;
-            int qsum = 0;
+            // q = rint(x * inv) (half to even), by the float adder: exact
+            // for |x * inv| < 2^22; inv = 0 (all-zero row) gives q = 0
+            int qi[4];
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
-                int qi = 0;
-                if (inv[m] > 0.0f) {
-                    qi = __float2int_rn(__fmul_rn(r[e], inv[m]));
-                    qi = max(-127, min(127, qi));
-                }
-                qsum += qi;
-                packed |= (static_cast<uint32_t>(qi) & 0xffu) << (8 * e);
+                const float t = __fadd_rn(__fmul_rn(r[e], inv[m]), 12582912.0f);
+                qi[e] = max(-127, min(127, __float_as_int(t) - 0x4B400000));
             }
-            qsum = __reduce_add_sync(0xffffffffu, qsum);  // one warp-wide reduction
+            const uint32_t packed =
+                __byte_perm(__byte_perm(qi[0], qi[1], 0x0040), __byte_perm(qi[2], qi[3], 0x0040), 0x5410);
+            const int qsum = __reduce_add_sync(0xffffffffu, dp4a_ss(packed, 0x01010101u, 0));
             *reinterpret_cast<uint32_t *>(act + m * L.Kpad + 128 * b + 4 * lane) = packed;
             if (lane == 0) sq[(m * L.GT + b) * 4] = qsum;
         };
