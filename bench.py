@@ -110,14 +110,36 @@ def prefill_gemm(fmt_id, Ms=(512, 2048, 8192), K=5120, N=17408, reps=10):
             "unit": "TOPS", "peak": peak, "peak_kind": kind, "results": res}
 
 
-def dist_setup(n_gpus):
+def dist_setup(n_gpus, backend="nccl"):
+    """One process per GPU (torch.distributed.run sets RANK / WORLD_SIZE /
+    LOCAL_RANK / MASTER_*).  The replicas share no data-path collective; the
+    process group only carries the barrier and the max-over-ranks timing.
+    A short timeout makes ranks that wait for a missing peer fail."""
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
     if world > 1:
         import torch.distributed as dist
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
     return world, rank, local
+
+
+def max_over_ranks(values, world, device="cuda"):
+    """Element-wise max of per-rank timings (every rank calls it, in the same
+    order); a single process returns them unchanged."""
+    if world <= 1:
+        return list(values)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor(list(values), dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return t.tolist()
+
+
+def replica_value(bytes_per_step, ms_per_step, world):
+    """Whole-job throughput of N weak-scaled replicas: every rank streams
+    bytes_per_step per step; the step time is the slowest rank's."""
+    return world * bytes_per_step / (ms_per_step * 1e-3) / 1e9
 
 
 class ClockSampler:
@@ -404,16 +426,12 @@ def main():
     e2e_ms = t2.elapsed_time(t3) / args.steps
     clk = clocks.stop()
 
-    if world > 1:
-        import torch.distributed as dist
-        t = torch.tensor([ms, e2e_ms, gu_ms], device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms, e2e_ms, gu_ms = t.tolist()
+    ms, e2e_ms, gu_ms = max_over_ranks([ms, e2e_ms, gu_ms], world)
 
     err = tern.tern_device_error()
     step_bytes = model.bytes_per_step()
-    value = world * step_bytes / (ms * 1e-3) / 1e9
-    e2e_val = world * step_bytes / (e2e_ms * 1e-3) / 1e9
+    value = replica_value(step_bytes, ms, world)
+    e2e_val = replica_value(step_bytes, e2e_ms, world)
     peak, peak_kind = peaks()
     gu_achieved = gu_bytes / (gu_ms * 1e-3) / 1e9
     out_ok = bool(torch.isfinite(model.x).all().item())
