@@ -47,6 +47,7 @@ constexpr int kGmWarps = 2 + kGmDecodeWarps + kGmEpiWarps;
 constexpr int kGmThreads = 32 * kGmWarps;
 constexpr int kGmAccBufs = 4;
 constexpr int kGmTmemCols = 128 * kGmAccBufs;  // four 128-column int32 accumulators
+constexpr int kGmBand = 8;                     // weight-row tiles per raster band
 constexpr int kGmEpiBar = 1;                   // named barrier of the epilogue warps
 
 struct GemmParams {
@@ -121,7 +122,16 @@ __global__ void __launch_bounds__(kGmThreads, 1)
     GemmSmem &S = *reinterpret_cast<GemmSmem *>(
         smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023));
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int n0 = blockIdx.x * kGmTileN, m0 = blockIdx.y * kGmTileM;
+    // Tile order: bands of kGmBand weight-row tiles, token tiles fastest
+    // inside a band, so the CTAs resident at one time cover a patch of about
+    // kGmBand x (148 / kGmBand) tiles: each activation tile is read by about
+    // kGmBand CTAs at once, not by every weight-row tile of the grid.
+    const int tiles_n = (p.N + kGmTileN - 1) / kGmTileN, tiles_m = (p.M + kGmTileM - 1) / kGmTileM;
+    const int band = blockIdx.x / (kGmBand * tiles_m);
+    const int band_w = min(kGmBand, tiles_n - band * kGmBand);
+    const int in_band = blockIdx.x - band * kGmBand * tiles_m;
+    const int n0 = (band * kGmBand + in_band % band_w) * kGmTileN;
+    const int m0 = (in_band / band_w) * kGmTileM;
     const int G = p.G;
     // After a failed wait anywhere (recorded in the device error word) the
     // remaining CTAs leave at once instead of timing out one by one.
@@ -339,8 +349,7 @@ cudaError_t launch_gemm(const GemmLaunch &L, cudaStream_t s, const char **why) {
     e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
     if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(static_cast<unsigned>(ceil_div(L.N, kGmTileN)),
-                       static_cast<unsigned>(ceil_div(L.M, kGmTileM)), 1);
+    cfg.gridDim = dim3(static_cast<unsigned>(ceil_div(L.N, kGmTileN) * ceil_div(L.M, kGmTileM)), 1, 1);
     cfg.blockDim = dim3(kGmThreads, 1, 1);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = s;
