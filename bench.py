@@ -193,7 +193,8 @@ class ClockSampler:
 
 def source_digest() -> str:
     h = hashlib.sha256()
-    for rel in ("ternary_weight_decode_b200/csrc/tern_gemv.cu",
+    for rel in ("ternary_weight_decode_b200/csrc/tern_gemv_stream.cu",
+                "ternary_weight_decode_b200/csrc/tern_gemv_common.cuh",
                 "ternary_weight_decode_b200/csrc/tern_common.cuh"):
         with open(os.path.join(ROOT, rel), "rb") as f:
             h.update(f.read())
