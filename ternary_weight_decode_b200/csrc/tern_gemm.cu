@@ -35,18 +35,20 @@ namespace tern {
 namespace {
 
 constexpr int kGmTileN = 128;   // weight rows per CTA (MMA M)
-constexpr int kGmTileM = 128;   // tokens per CTA (MMA N)
-constexpr int kGmTile = 128 * 128;  // bytes of one 128 x 128 B int8 tile
+constexpr int kGmTileM = 256;   // tokens per CTA (MMA N)
+constexpr int kGmTile = 128 * 128;  // bytes of one 128 x 128 B int8 tile (codes, decoded A)
+constexpr int kGmActTile = kGmTileM * 128;  // bytes of one activation tile (kGmTileM x 128 B)
 constexpr int kGmCodeStages = 2;
-constexpr int kGmActStages = 4;
+constexpr int kGmActStages = 3;
 constexpr int kGmAStages = 2;
-constexpr int kGmDecodeWarps = 8;
-constexpr int kGmEpiWarps = 8;
+constexpr int kGmDecodeWarps = 4;
+constexpr int kGmEpiWarps = 16;
 constexpr int kGmEpiCols = kGmTileM * 4 / kGmEpiWarps;  // token columns per epilogue warp
 constexpr int kGmWarps = 2 + kGmDecodeWarps + kGmEpiWarps;
 constexpr int kGmThreads = 32 * kGmWarps;
-constexpr int kGmAccBufs = 4;
-constexpr int kGmTmemCols = 128 * kGmAccBufs;  // four 128-column int32 accumulators
+constexpr int kGmAccBufs = 2;
+constexpr int kGmTmemCols = kGmTileM * kGmAccBufs;  // kGmAccBufs accumulators of kGmTileM columns
+static_assert(kGmTmemCols <= 512, "tensor memory holds 512 columns");
 constexpr int kGmBand = 8;                     // weight-row tiles per raster band
 constexpr int kGmEpiBar = 1;                   // named barrier of the epilogue warps
 
@@ -60,7 +62,7 @@ struct GemmParams {
 
 struct GemmSmem {
     uint8_t code[kGmCodeStages][kGmTile];
-    uint8_t act[kGmActStages][kGmTile];
+    uint8_t act[kGmActStages][kGmActTile];
     uint8_t a[kGmAStages][kGmTile];
     uint64_t code_full[kGmCodeStages], code_empty[kGmCodeStages];
     uint64_t act_full[kGmActStages], act_empty[kGmActStages];
@@ -185,7 +187,7 @@ __global__ void __launch_bounds__(kGmThreads, 1)
                     if (g >= kGmActStages &&
                         !mbar_wait_bounded(&S.act_empty[as], ((g / kGmActStages) - 1) & 1))
                         break;
-                    mbar_arrive_expect_tx(&S.act_full[as], kGmTile);
+                    mbar_arrive_expect_tx(&S.act_full[as], kGmActTile);
                     tma_load_2d_nohint(S.act[as], &tm_q, g * 128, m0, &S.act_full[as]);
                 }
             }
@@ -205,7 +207,7 @@ __global__ void __launch_bounds__(kGmThreads, 1)
                 const uint32_t a0 = smem_u32(S.a[as]), b0 = smem_u32(S.act[qs]);
 #pragma unroll
                 for (int s = 0; s < 4; ++s)
-                    mma_i8_ss(tmem + buf * 128, smem_desc_sw128(a0 + 32 * s),
+                    mma_i8_ss(tmem + buf * kGmTileM, smem_desc_sw128(a0 + 32 * s),
                               smem_desc_sw128(b0 + 32 * s), idesc, s > 0);
                 tc_commit(&S.acc_full[buf]);
                 tc_commit(&S.a_empty[as]);
@@ -244,10 +246,14 @@ __global__ void __launch_bounds__(kGmThreads, 1)
                                 mbar_wait_bounded(&S.a_empty[as], ((g / kGmAStages) - 1) & 1)))
                     break;
                 uint8_t *arow = S.a[as] + r * 128;
-                if (half == 0)
-                    decode_half<FMT, 0>(words, gg, arow, r);
-                else
+                if constexpr (kGmDecodeWarps == 4) {
+                    decode_half<FMT, 0>(words, gg, arow, r);  // a thread = one row, whole group
                     decode_half<FMT, 1>(words, gg, arow, r);
+                } else if (half == 0) {
+                    decode_half<FMT, 0>(words, gg, arow, r);
+                } else {
+                    decode_half<FMT, 1>(words, gg, arow, r);
+                }
                 fence_proxy_async_smem();  // read by the tensor cores
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&S.a_full[as]);
@@ -256,7 +262,7 @@ __global__ void __launch_bounds__(kGmThreads, 1)
         }
     } else {
         // -------------------------------------------------------- epilogue
-        const int e = warp - 2 - kGmDecodeWarps;      // 0..7
+        const int e = warp - 2 - kGmDecodeWarps;      // 0 .. kGmEpiWarps-1
         const int quarter = warp & 3;                  // tensor-memory lanes it reaches
         const int c0 = (e >> 2) * kGmEpiCols;         // its token columns
         const int r = 32 * quarter + lane;             // tile row
@@ -279,19 +285,19 @@ __global__ void __launch_bounds__(kGmThreads, 1)
                 __all_sync(0xffffffffu, mbar_wait_bounded(&S.acc_full[buf], (g / kGmAccBufs) & 1));
             if (!ok) break;
             tc_fence_after_sync();
-            uint32_t v[16];
+            uint32_t v[8];
 #pragma unroll
-            for (int h = 0; h < kGmEpiCols / 16; ++h) {
-                tmem_ld16(tmem + lane_addr + buf * 128 + c0 + 16 * h, v);
+            for (int h = 0; h < kGmEpiCols / 8; ++h) {
+                tmem_ld8(tmem + lane_addr + buf * kGmTileM + c0 + 8 * h, v);
                 tmem_wait_ld();
-                if (h == kGmEpiCols / 16 - 1) {
+                if (h == kGmEpiCols / 8 - 1) {
                     tc_fence_before_sync();
                     __syncwarp();
                     if (lane == 0) mbar_arrive(&S.acc_empty[buf]);
                 }
 #pragma unroll
-                for (int c = 0; c < 16; ++c)
-                    acc[16 * h + c] = fmaf(s, __int2float_rn(static_cast<int>(v[c])), acc[16 * h + c]);
+                for (int c = 0; c < 8; ++c)
+                    acc[8 * h + c] = fmaf(s, __int2float_rn(static_cast<int>(v[c])), acc[8 * h + c]);
             }
         }
         pdl_wait();  // s_x comes from the previous kernel
