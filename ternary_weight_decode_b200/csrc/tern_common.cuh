@@ -21,6 +21,8 @@ enum : int {
 
 // Budget of a bounded wait, in SM clock cycles (about 0.5 s at 2 GHz).
 constexpr long long kWaitBudgetCycles = 1000000000LL;
+// Back-off between polls of a wait that is not yet satisfied (ns).
+constexpr unsigned kWaitBackoffNs = 32;
 
 __device__ __forceinline__ uint32_t smem_u32(const void *p) {
     return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -64,6 +66,7 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint64_t *bar, uint32_t parity
     if (mbar_try_wait(bar, parity)) return true;
     long long start = clock64();
     while (!mbar_try_wait(bar, parity)) {
+        __nanosleep(kWaitBackoffNs);  // leave the issue slots to warps with work
         if (clock64() - start > kWaitBudgetCycles) {
             atomicExch(&g_device_error, kErrTmaTimeout);
             return false;
@@ -214,6 +217,7 @@ __device__ __forceinline__ bool mbar_wait_cluster_bounded(uint64_t *bar, uint32_
     if (mbar_try_wait_cluster(bar, parity)) return true;
     long long start = clock64();
     while (!mbar_try_wait_cluster(bar, parity)) {
+        __nanosleep(kWaitBackoffNs);
         if (clock64() - start > kWaitBudgetCycles) {
             atomicExch(&g_device_error, kErrTmaTimeout);
             return false;

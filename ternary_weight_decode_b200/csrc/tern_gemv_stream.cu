@@ -672,6 +672,7 @@ __global__ void __launch_bounds__(kSkThreads, 2)
                         if ((w >> 32) == 0) {
                             const long long start = clock64();
                             while (((w = ld_relaxed_gpu_u64(t)) >> 32) == 0) {
+                                __nanosleep(kWaitBackoffNs);
                                 if (clock64() - start > kWaitBudgetCycles) {
                                     atomicExch(&g_device_error, kErrTmaTimeout);
                                     break;
