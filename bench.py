@@ -473,7 +473,9 @@ def main():
         "bytes_per_step": step_bytes,
         "e2e": {"value": e2e_val, "unit": "GB/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "tok_s_equiv": world * 1e3 / e2e_ms},
-        "roofline": {"bound": "hbm", "kernel": "tern_gateup_swiglu (fused gate/up + SwiGLU, K=5120, N=17408)",
+        "roofline": {"bound": "hbm",
+                     "kernel": f"tern_gateup_swiglu{'_streamed' if mode == 'streamed' else '_fused' if mode == 'fused' else ''}"
+                               " (gate/up + SwiGLU, K=5120, N=17408, 2 matrices)",
                      "achieved": gu_achieved, "peak": peak, "peak_kind": peak_kind, "unit": "GB/s",
                      "frac": gu_achieved / peak, "traffic": traffic_record("gateup_swiglu", args.fmt),
                      "algorithmic_bytes_per_launch": gu_bytes, "avg_launch_us": gu_ms * 1e3},
