@@ -69,13 +69,21 @@ __host__ __device__ constexpr int align128(int v) { return (v + 127) & ~127; }
 // with the activation word at K = 20w + 4i): a code byte y = ceil(256 V/243)
 // gives D_i = floor(y 3^(i+1) / 256).  Two bytes share one 32-bit multiply
 // (16-bit lanes, y 3^(i+1) < 2^16); PRMT gathers the four high bytes.
+// 3 z as a shift and an add: integer ALU work, leaving the multiply pipe
+// (shared with dp4a) to the dot product.  Exact: 3 z = z + 2 z mod 2^32.
+__device__ __forceinline__ uint32_t times3(uint32_t z) {
+    uint32_t r;
+    asm("{\n\t.reg .u32 t;\n\tshl.b32 t, %1, 1;\n\tadd.u32 %0, t, %1;\n\t}" : "=r"(r) : "r"(z));
+    return r;
+}
+
 __device__ __forceinline__ void decode_d3_D(uint32_t X, uint32_t (&D)[5]) {
     uint32_t ze = X & 0x00FF00FFu;         // bytes 0 and 2
     uint32_t zo = (X >> 8) & 0x00FF00FFu;  // bytes 1 and 3
 #pragma unroll
     for (int i = 0; i < 5; ++i) {
-        ze *= 3u;
-        zo *= 3u;
+        ze = times3(ze);
+        zo = times3(zo);
         D[i] = __byte_perm(ze, zo, 0x7351);
     }
 }
