@@ -772,6 +772,13 @@ cudaError_t launch_sk(const StreamLaunch &S, cudaStream_t s, const char **why) {
     if (!plan_c[dev]) {
         e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
         if (e != cudaSuccess) return e;
+        // Every launch takes the largest shared-memory split of the SM, so
+        // that a launch waiting on its predecessor (programmatic launch) can
+        // sit beside it on the same SM: launches whose splits differ cannot
+        // share an SM, which then drains before the next one starts.
+        e = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                 cudaSharedmemCarveoutMaxShared);
+        if (e != cudaSuccess) return e;
         plan_c[dev] = choose_cluster(kern, S.num_sms, &plan_n[dev]);
     }
     // The smallest cluster whose CTAs hold their share of the input blocks in
