@@ -23,10 +23,11 @@
 //    sends it to every CTA of the cluster (st.async into their shared
 //    memory), then quantises its blocks with the cluster-wide row scale and
 //    sends the int8 codes and group sums to every CTA the same way.
-//  * Consumers then take items round-robin: lane = row; the item's codes and
-//    scales are copied to registers and the ring slot is handed back at once,
-//    so the whole ring stays in flight; decode + dp4a as in tern_gemv.cu; one
-//    fp32 partial per (item, row, token).
+//  * Consumers then take items round-robin: lane = row; decode + dp4a as in
+//    tern_gemv.cu; one fp32 partial per (item, row, token).  A 2-bit item is
+//    copied to registers and its ring slot handed back at once, so the whole
+//    ring stays in flight; a base-3 item, whose decode outlasts the refill of
+//    a slot, is read from the slot as it is decoded and handed back after.
 //  * Row blocks inside a CTA's range are summed in unit order and written.
 //    A row block cut by a range boundary belongs to two CTAs.  The one that
 //    holds its end (its first units) publishes its partial as soon as those
@@ -44,12 +45,13 @@ namespace {
 constexpr int kSkConsumers = 8;
 constexpr int kSkThreads = 32 * (kSkConsumers + 1);
 constexpr int kSkBar = 1;   // named barrier of the consumer warps
-// Input blocks a consumer warp keeps in registers between the two passes
-// (one token row: K up to 9 x 8 warps x 2 CTAs x 128 = 18432 without reloads).
-template <int MT>
-__host__ __device__ constexpr int sk_keep() {
-    return MT == 1 ? 9 : 5;
-}
+// Input blocks a consumer warp loads at once (one round) and keeps in
+// registers between the two passes: a K of 5 x 8 warps x 128 = 5120 per CTA
+// is one round; a longer share takes several, the earlier ones loaded again
+// for the second pass.  The prologue is unrolled over a round and runs once
+// per launch: rounds of 9 (one round up to K = 18432 with clusters of 2)
+// measured slower, their code costing more than the reloads they save.
+constexpr int kSkKeep = 5;
 constexpr int kSkMaxCluster = 4;
 constexpr int kSkSmemBudget = 112 * 1024;  // two CTAs per SM (programmatic launch overlap)
 constexpr int kSkMinRing = 8, kSkMaxRing = 24;  // unit slots, multiples of kSkChunk
@@ -121,14 +123,14 @@ __device__ __forceinline__ void bulk_copy_g2s(void *dst, const void *src, uint32
         : "memory");
 }
 
-// One item (this lane's row, one superblock of one matrix) from registers:
-// the decode and dp4a of tern_gemv.cu.  words: the row's 128 code bytes in
-// K order; sc: the row's GPS group scales; sq_sb: group sums of the input,
-// one per 4 ints.
-template <int FMT, int MT>
-__device__ __forceinline__ void sk_item(const uint32_t (&words)[32],
-                                        const float (&sc)[Fmt<FMT>::kGroups], const uint8_t *act_sb,
-                                        int Kpad, const int *sq_sb, int GT, float (&yacc)[MT]) {
+// One item (this lane's row, one superblock of one matrix): the decode and
+// dp4a of tern_gemv.cu.  words4(c): the row's code words 4c .. 4c+3 (bytes
+// 16c .. 16c+15 of its 128, K order); sc: the row's GPS group scales; sq_sb:
+// group sums of the input, one per 4 ints.
+template <int FMT, int MT, typename Words4>
+__device__ __forceinline__ void sk_item(Words4 words4, const float (&sc)[Fmt<FMT>::kGroups],
+                                        const uint8_t *act_sb, int Kpad, const int *sq_sb, int GT,
+                                        float (&yacc)[MT]) {
     int acc[MT];
 #pragma unroll
     for (int m = 0; m < MT; ++m) {
@@ -141,12 +143,14 @@ __device__ __forceinline__ void sk_item(const uint32_t (&words)[32],
     };
 #pragma unroll
     for (int c = 0; c < 8; ++c) {
+        const uint4 wv = words4(c);
+        const uint32_t words[4] = {wv.x, wv.y, wv.z, wv.w};
         if constexpr (FMT == TERN_FMT_BASE3) {
             uint32_t t[20];
 #pragma unroll
             for (int wi = 0; wi < 4; ++wi) {
                 uint32_t tw[5];
-                decode_d3(words[4 * c + wi], tw);
+                decode_d3(words[wi], tw);
 #pragma unroll
                 for (int i = 0; i < 5; ++i) t[5 * wi + i] = tw[i];
             }
@@ -187,8 +191,7 @@ __device__ __forceinline__ void sk_item(const uint32_t (&words)[32],
                 for (int wi = 0; wi < 4; ++wi)
 #pragma unroll
                     for (int i = 0; i < 4; ++i)
-                        a4[i] = dp4a_us(words[4 * c + wi] & (0x03030303u << (2 * i)), aw[4 * wi + i],
-                                        a4[i]);
+                        a4[i] = dp4a_us(words[wi] & (0x03030303u << (2 * i)), aw[4 * wi + i], a4[i]);
                 acc[m] += a4[0] + (a4[1] >> 2) + (a4[2] >> 4) + (a4[3] >> 6);
                 if (c & 1) finish(m, c >> 1);
             }
@@ -262,7 +265,7 @@ __global__ void __launch_bounds__(kSkThreads, 2)
                        const __grid_constant__ CUtensorMap tm3_1, const SkParams p) {
     constexpr int NMAT = (MODE == kModeSwiglu) ? 2 : 1;
     constexpr int CH = kSkChunk / NMAT;  // units of one matrix per ring chunk
-    constexpr int KEEP = sk_keep<MT>();
+    constexpr int KEEP = kSkKeep;
     constexpr int POS = Fmt<FMT>::kPos;
     constexpr int GPS = Fmt<FMT>::kGroups;
     constexpr int SCB = scb<FMT>();
@@ -399,51 +402,55 @@ __global__ void __launch_bounds__(kSkThreads, 2)
         const bool rotate = (p.qflags & TERN_QUANT_FWHT128) != 0;
         const bool rms = (p.qflags & TERN_QUANT_RMSNORM) != 0;
 
-        // pass 1: loads first (KEEP blocks per warp in flight), then the
-        // rotation, max |.| and sum x^2 of this CTA's blocks
+        // The warp's blocks of this CTA's share are b_lo + cw + 8 (KEEP r + j),
+        // taken in rounds r of KEEP.  A round's full 4-value loads are all
+        // issued before any is used (predicated volatile loads: the compiler
+        // may not interleave them with their uses); a block ending past K is
+        // read by load_block afterwards.
         float v[MT][KEEP][4];
+        auto blk = [&](int r, int j) { return b_lo + cw + kSkConsumers * (KEEP * r + j); };
+        auto load_round = [&](int r) {
+#pragma unroll
+            for (int m = 0; m < MT; ++m)
+#pragma unroll
+                for (int j = 0; j < KEEP; ++j) {
+                    const int b = blk(r, j);
+                    const int k = 128 * b + 4 * lane;
+                    const bool full = b < b_hi && m < p.M && k + 4 <= p.K;
+                    ld_cg_f32x4_pred(p.x + static_cast<int64_t>(m) * p.ldx + k, full, v[m][j]);
+                }
+#pragma unroll
+            for (int m = 0; m < MT; ++m)
+#pragma unroll
+                for (int j = 0; j < KEEP; ++j) {
+                    const int b = blk(r, j);
+                    const int k = 128 * b + 4 * lane;
+                    if (b < b_hi && m < p.M && k < p.K && k + 4 > p.K) load_block(p, m, b, lane, v[m][j]);
+                }
+        };
+        const int nblk = b_hi > b_lo + cw ? (b_hi - b_lo - cw + kSkConsumers - 1) / kSkConsumers : 0;
+        const int nrounds = nblk > KEEP ? (nblk + KEEP - 1) / KEEP : 1;
+
+        // pass 1: the rotation, max |.| and sum x^2 of the warp's blocks; the
+        // last round stays in registers
         float amax[MT], ss[MT];
-        // Every full 4-value load is issued before any is used (predicated
-        // volatile loads: the compiler may not interleave them with their
-        // uses); a block ending past K is read by load_block afterwards.
 #pragma unroll
         for (int m = 0; m < MT; ++m) {
             amax[m] = 0.0f;
             ss[m] = 0.0f;
-#pragma unroll
-            for (int j = 0; j < KEEP; ++j) {
-                const int b = b_lo + cw + kSkConsumers * j;
-                const int k = 128 * b + 4 * lane;
-                const bool full = b < b_hi && m < p.M && k + 4 <= p.K;
-                ld_cg_f32x4_pred(p.x + static_cast<int64_t>(m) * p.ldx + k, full, v[m][j]);
-            }
         }
+#pragma unroll 1
+        for (int r = 0; r < nrounds; ++r) {
+            load_round(r);
 #pragma unroll
-        for (int m = 0; m < MT; ++m)
+            for (int m = 0; m < MT; ++m)
 #pragma unroll
-            for (int j = 0; j < KEEP; ++j) {
-                const int b = b_lo + cw + kSkConsumers * j;
-                const int k = 128 * b + 4 * lane;
-                if (b < b_hi && m < p.M && k < p.K && k + 4 > p.K) load_block(p, m, b, lane, v[m][j]);
-            }
-#pragma unroll
-        for (int m = 0; m < MT; ++m)
-#pragma unroll
-            for (int j = 0; j < KEEP; ++j) {
-                if (b_lo + cw + kSkConsumers * j >= b_hi) continue;
-                ss[m] += sumsq4(v[m][j]);
-                if (rotate) fwht128_warp(v[m][j], lane);
-                amax[m] = fmaxf(amax[m], amax4(v[m][j]));
-            }
-        for (int b = b_lo + cw + kSkConsumers * KEEP; b < b_hi; b += kSkConsumers) {
-#pragma unroll
-            for (int m = 0; m < MT; ++m) {
-                float r[4];
-                load_block(p, m, b, lane, r);
-                ss[m] += sumsq4(r);
-                if (rotate) fwht128_warp(r, lane);
-                amax[m] = fmaxf(amax[m], amax4(r));
-            }
+                for (int j = 0; j < KEEP; ++j) {
+                    if (blk(r, j) >= b_hi) continue;
+                    ss[m] += sumsq4(v[m][j]);
+                    if (rotate) fwht128_warp(v[m][j], lane);
+                    amax[m] = fmaxf(amax[m], amax4(v[m][j]));
+                }
         }
 #pragma unroll
         for (int m = 0; m < MT; ++m) {
@@ -529,21 +536,27 @@ __global__ void __launch_bounds__(kSkThreads, 2)
             *reinterpret_cast<uint32_t *>(act + m * L.Kpad + 128 * b + 4 * lane) = packed;
             if (lane == 0) sq[(m * L.GT + b) * 4] = qsum;
         };
+        // the last round from registers; earlier ones loaded again, a round
+        // at a time
 #pragma unroll
         for (int m = 0; m < MT; ++m)
 #pragma unroll
             for (int j = 0; j < KEEP; ++j) {
-                const int b = b_lo + cw + kSkConsumers * j;
+                const int b = blk(nrounds - 1, j);
                 if (b < b_hi) quant_block(m, b, v[m][j]);
             }
-        for (int b = b_lo + cw + kSkConsumers * KEEP; b < b_hi; b += kSkConsumers) {
+#pragma unroll 1
+        for (int r = 0; r + 1 < nrounds; ++r) {
+            load_round(r);
 #pragma unroll
-            for (int m = 0; m < MT; ++m) {
-                float r[4];
-                load_block(p, m, b, lane, r);
-                if (rotate) fwht128_warp(r, lane);
-                quant_block(m, b, r);
-            }
+            for (int m = 0; m < MT; ++m)
+#pragma unroll
+                for (int j = 0; j < KEEP; ++j) {
+                    const int b = blk(r, j);
+                    if (b >= b_hi) continue;
+                    if (rotate) fwht128_warp(v[m][j], lane);
+                    quant_block(m, b, v[m][j]);
+                }
         }
         fence_proxy_async_smem();  // the share is read by the bulk copies
         warpgroup_sync_n(kSkBar, kSkConsumers * 32);
@@ -568,7 +581,7 @@ __global__ void __launch_bounds__(kSkThreads, 2)
         // same position in a chunk, hence the same matrix); the item is copied
         // to registers and its chunk slot handed back at once.  Chunk, phase
         // and superblock advance incrementally (two chunks a step).
-        const int pos = cw % kSkChunk, mat_w = pos / CH, uoff = pos % CH;
+        const int pos = cw % kSkChunk, uoff = pos % CH;
         int kc = cw / kSkChunk;
         int kcs = kc % RC, phase = (kc / RC) & 1;
         int sb = static_cast<int>((u0 + kc * CH + uoff) % p.SB);
@@ -582,25 +595,33 @@ __global__ void __launch_bounds__(kSkThreads, 2)
             const int slot = kcs * kSkChunk + pos;
             float yacc[MT];
             if (ok) {
-                uint32_t words[32];
+                // the lane's row of the slot: 8 chunks of 16 bytes, 128-byte swizzle
                 const uint8_t *wt = ring_w + slot * kTile + lane * kSBBytes;
                 const int rsw = lane & 7;
-#pragma unroll
-                for (int cc = 0; cc < 8; ++cc) {
-                    const uint4 wv = lds128(wt + ((cc ^ rsw) << 4));
-                    words[4 * cc + 0] = wv.x;
-                    words[4 * cc + 1] = wv.y;
-                    words[4 * cc + 2] = wv.z;
-                    words[4 * cc + 3] = wv.w;
-                }
                 float sc[GPS];
                 const uint16_t *st =
                     reinterpret_cast<const uint16_t *>(ring_s + slot * SCB) + lane * GPS;
 #pragma unroll
                 for (int g = 0; g < GPS; ++g) sc[g] = __half2float(__ushort_as_half(st[g]));
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&empty[kcs]);
-                sk_item<FMT, MT>(words, sc, act + sb * POS, L.Kpad, sq + sb * GPS * 4, L.GT, yacc);
+                if constexpr (FMT == TERN_FMT_BASE3) {
+                    // The decode takes longer than the slot takes to refill:
+                    // the words are read from the slot as they are used
+                    // (fewer live registers for the decode), and the slot is
+                    // handed back when the item is done.
+                    sk_item<FMT, MT>([&](int cc) { return lds128(wt + ((cc ^ rsw) << 4)); }, sc,
+                                     act + sb * POS, L.Kpad, sq + sb * GPS * 4, L.GT, yacc);
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&empty[kcs]);
+                } else {
+                    // copied to registers, the slot handed back at once
+                    uint4 wv[8];
+#pragma unroll
+                    for (int cc = 0; cc < 8; ++cc) wv[cc] = lds128(wt + ((cc ^ rsw) << 4));
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&empty[kcs]);
+                    sk_item<FMT, MT>([&](int cc) { return wv[cc]; }, sc, act + sb * POS, L.Kpad,
+                                     sq + sb * GPS * 4, L.GT, yacc);
+                }
             } else {
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&empty[kcs]);
@@ -785,7 +806,7 @@ cudaError_t launch_sk(const StreamLaunch &S, cudaStream_t s, const char **why) {
     // registers (no reloads); a single CTA needs no exchange at all.
     const int GT = p.SB * Fmt<FMT>::kGroups;
     int C = 1;
-    while (C < plan_c[dev] && ceil_div(ceil_div(GT, C), kSkConsumers) > sk_keep<MT>()) C *= 2;
+    while (C < plan_c[dev] && ceil_div(ceil_div(GT, C), kSkConsumers) > kSkKeep) C *= 2;
     // every range holds >= SB units, so a row block meets at most 2 ranges
     long long want = p.U / p.SB;
     if (want > (C > 1 ? plan_n[dev] : S.num_sms)) want = C > 1 ? plan_n[dev] : S.num_sms;
