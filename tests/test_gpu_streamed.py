@@ -26,7 +26,11 @@ def leftovers(ws):
 @pytest.mark.parametrize("fmt", FMTS)
 @pytest.mark.parametrize("N,K,M,qflags", [(256, 256, 1, 0), (7168, 5120, 1, RMS), (5120, 17408, 1, RMS),
                                           (5120, 5120, 2, ROT), (37, 300, 1, 0), (1000, 1280, 2, RMS | ROT),
-                                          (33, 20, 1, 0), (4100, 17408, 2, 0)])
+                                          (33, 20, 1, 0), (4100, 17408, 2, 0),
+                                          # several rounds of input blocks per warp: rotated (K % 128
+                                          # == 0), a partial last block, three rounds
+                                          (1000, 17408, 1, RMS | ROT), (700, 17407, 2, RMS),
+                                          (600, 29952, 1, RMS | ROT), (300, 30001, 2, RMS)])
 def test_streamed_gemv_matches_oracle(fmt, N, K, M, qflags):
     w = synth.trits(31, 0, N, K)
     sw = synth.scales(31, 1, N, synth.groups(K))
@@ -50,14 +54,18 @@ def test_streamed_gemv_matches_oracle(fmt, N, K, M, qflags):
 
 
 @pytest.mark.parametrize("fmt", FMTS)
-@pytest.mark.parametrize("N,K,M", [(17408, 5120, 1), (17408, 5120, 2), (300, 640, 1)])
+@pytest.mark.parametrize("N,K,M", [(17408, 5120, 1), (17408, 5120, 2), (300, 640, 1),
+                                   (600, 12800, 1), (260, 17408, 2)])
 def test_streamed_gateup(fmt, N, K, M):
     wg, wu = synth.trits(32, 4, N, K), synth.trits(32, 6, N, K)
     G = synth.groups(K)
     sg, su = synth.scales(32, 5, N, G), synth.scales(32, 7, N, G)
     Wg, Wu = tiled(fmt, wg, sg), tiled(fmt, wu, su)
     xh = synth.activation_rows(range(70, 70 + M), K).astype(np.float32)
-    x = to_dev(xh)
+    ldx = ((K + 3) // 4) * 4  # rows 16-byte aligned; the columns past K are not read
+    xb = np.full((M, ldx), np.nan, np.float32)
+    xb[:, :K] = xh
+    x = to_dev(xb)[:, :K]
     ws = tern.stream_workspace(fmt, N, M, True)
     h = torch.zeros((M, N), dtype=torch.float32, device="cuda")
     tern.tern_gateup_swiglu_streamed(Wg, Wu, x, h, ws, qflags=RMS | ROT)
