@@ -405,6 +405,12 @@ cudaError_t launch_cc(const GemvLaunch &Lh, cudaStream_t s, const char **why) {
         e = cudaFuncSetAttribute(gemv_cc_kernel<FMT, MT, MODE, XIN>,
                                  cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
         if (e != cudaSuccess) return e;
+        // The largest shared-memory split for every launch, so that a launch
+        // waiting on its predecessor (programmatic launch) can share its SMs:
+        // launches whose splits differ cannot, and the SM drains first.
+        e = cudaFuncSetAttribute(gemv_cc_kernel<FMT, MT, MODE, XIN>,
+                                 cudaFuncAttributePreferredSharedMemoryCarveout, cudaSharedmemCarveoutMaxShared);
+        if (e != cudaSuccess) return e;
         smem_set[dev] = 1;
     }
     cudaLaunchConfig_t cfg = {};
