@@ -84,6 +84,10 @@ def _load():
             lib.oracle_swiglu.argtypes = [p, p, i64, p]
             lib.oracle_gateup_swiglu.restype = i32
             lib.oracle_gateup_swiglu.argtypes = [p, p, p, p, i64, i64, i64, p, p, i64, p]
+            lib.oracle_float_to_half.restype = ctypes.c_uint16
+            lib.oracle_float_to_half.argtypes = [ctypes.c_float]
+            lib.oracle_ternarize.restype = i32
+            lib.oracle_ternarize.argtypes = [p, i64, i64, i64, i64, p, p]
             _lib = lib
     return _lib
 
@@ -266,3 +270,22 @@ def gateup_swiglu(wg, sg, wu, su, q, s_x, group: int = 128) -> np.ndarray:
     _check(_load().oracle_gateup_swiglu(_ptr(wg), _ptr(sg), _ptr(wu), _ptr(su), N, K, group,
                                         _ptr(q), _ptr(s_x), M, _ptr(h)), "gateup_swiglu")
     return h
+
+
+# ---------------------------------------------------------------- ternarisation
+def float_to_half_bits(f: float) -> int:
+    """IEEE binary16 bits of fp32 f, round to nearest even."""
+    return int(_load().oracle_float_to_half(float(np.float32(f))))
+
+
+def ternarize(w: np.ndarray, group: int = 128):
+    """(trits int8 [N, K], scales float16 [N, G]) of fp32 weights w [N, K]:
+    per group the MSE-optimal symmetric thresholds and scale, in the fp32
+    arithmetic the C file states (its reading R10)."""
+    w = _c(w, np.float32)
+    N, K = w.shape
+    G = groups(K, group)
+    t = np.zeros((N, K), np.int8)
+    sc = np.zeros((N, G), np.uint16)
+    _check(_load().oracle_ternarize(_ptr(w), N, K, K, group, _ptr(t), _ptr(sc)), "ternarize")
+    return t, sc.view(np.float16)

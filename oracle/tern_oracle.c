@@ -46,6 +46,20 @@
  *  R9 decode chain glue (the pages give no norm or attention detail): a
  *     weightless RMSNorm of the unrotated row folded into the scale only,
  *     s_x / sqrt(mean(x^2) + 1e-6), which leaves every int8 code unchanged.
+ *  R10 ternarisation (pwwt.cn/news/5175886, section 1.2: per block, two
+ *     thresholds -- values between them become 0, the two sides +1 / -1 --
+ *     and a scale chosen to make the residual small; m.nxbn.cn/news/172464,
+ *     section 1.2: threshold plus one scale per group; no calibration data
+ *     here, so the residual is that of the weights themselves).  Per group of
+ *     128 consecutive K positions of a row: the thresholds are -D and +D and
+ *     the scale alpha is the one that minimises sum (w - alpha t)^2, i.e.
+ *     keep the k largest |w| (ties: lower index first) for the k that
+ *     maximises S_k^2 / k, S_k = their sum.  Arithmetic fixed in fp32 so
+ *     that the integer decisions are reproducible: S_k is the fp32 sum of
+ *     the kept |w| in index order, score = fp32(fp32(S_k * S_k) / k), the
+ *     largest score wins and among equal scores the smallest k (k = 0,
+ *     score 0, when nothing beats it); alpha = fp16(fp32(S_k / k)), rounded
+ *     to nearest even.
  *
  * Device layouts (the "load-time retile into consumption order" suggested on
  * [BONSAI], section "后面还有没有优化空间"):
@@ -405,4 +419,88 @@ int oracle_gateup_swiglu(const int8_t *wg, const uint16_t *sg, const int8_t *wu,
     free(g);
     free(u);
     return rc;
+}
+
+/* ------------------------------------------------------------------ */
+/* fp32 -> IEEE binary16 bits, round to nearest, ties to even, written from
+ * the format's definition: 1 sign bit, 5 exponent bits (bias 15), 10
+ * fraction bits; subnormals below 2^-14; overflow to infinity.           */
+uint16_t oracle_float_to_half(float f) {
+    uint32_t x;
+    memcpy(&x, &f, 4);
+    uint16_t sign = (uint16_t)((x >> 16) & 0x8000u);
+    uint32_t e = (x >> 23) & 0xffu;
+    uint32_t m = x & 0x7fffffu;
+    if (e == 0xffu) return (uint16_t)(sign | 0x7c00u | (m ? 0x200u : 0u)); /* inf / nan */
+    double a = fabs((double)f);                        /* exact */
+    if (a == 0.0) return sign;
+    /* value = a = q * 2^E with the fp16 quantum of a's binade */
+    int ex;
+    frexp(a, &ex);                                     /* a = f * 2^ex, f in [0.5, 1) */
+    int E = ex - 1;                                    /* a in [2^E, 2^(E+1)) */
+    if (E < -14) E = -14;                              /* subnormal range: quantum 2^-24 */
+    double quantum = ldexp(1.0, E - 10);
+    double qv = a / quantum;                           /* exact (power-of-two scaling) */
+    double r = floor(qv);
+    double rem = qv - r;
+    if (rem > 0.5 || (rem == 0.5 && fmod(r, 2.0) != 0.0)) r += 1.0;
+    double v = r * quantum;                            /* rounded magnitude */
+    if (v >= 65520.0 || v > 65504.0) return (uint16_t)(sign | 0x7c00u);
+    /* encode v */
+    if (v < ldexp(1.0, -14)) return (uint16_t)(sign | (uint16_t)(v / ldexp(1.0, -24)));
+    frexp(v, &ex);
+    E = ex - 1;
+    uint32_t frac = (uint32_t)(v / ldexp(1.0, E - 10)) - 1024u;
+    return (uint16_t)(sign | (uint16_t)((E + 15) << 10) | (uint16_t)frac);
+}
+
+/* Ternarisation of one matrix (R10).  w: fp32 [N][K] (finite), row stride
+ * ldw; t: int8 [N][K] in {-1,0,+1}; scales: fp16 bits [N][ceil(K/group)]. */
+int oracle_ternarize(const float *w, int64_t N, int64_t K, int64_t ldw, int64_t group,
+                     int8_t *t, uint16_t *scales) {
+    if (group <= 0 || ldw < K) return ORACLE_EINVAL;
+    int64_t G = oracle_groups(K, group);
+    for (int64_t n = 0; n < N; ++n) {
+        for (int64_t g = 0; g < G; ++g) {
+            int64_t k0 = g * group, k1 = (g + 1) * group < K ? (g + 1) * group : K;
+            const float *v = w + n * ldw;
+            /* candidate j keeps every i ranked at or above j: |w_i| > |w_j|,
+             * or |w_i| == |w_j| with i <= j; it keeps cnt(j) = rank(j) + 1 */
+            int64_t best_cnt = 0;
+            float best_score = 0.0f, best_sum = 0.0f;
+            for (int64_t j = k0; j < k1; ++j) {
+                float aj = fabsf(v[j]);
+                volatile float sum = 0.0f;
+                int64_t cnt = 0;
+                for (int64_t i = k0; i < k1; ++i) {
+                    float ai = fabsf(v[i]);
+                    if (ai > aj || (ai == aj && i <= j)) {
+                        sum = sum + ai;
+                        ++cnt;
+                    }
+                }
+                volatile float sq = sum * sum;
+                volatile float score = sq / (float)cnt;
+                if (score > best_score || (score == best_score && cnt < best_cnt)) {
+                    best_score = score;
+                    best_cnt = cnt;
+                    best_sum = sum;
+                }
+            }
+            /* keep the best_cnt largest |w| (same rank order) */
+            for (int64_t i = k0; i < k1; ++i) {
+                int64_t rank = 0;
+                float ai = fabsf(v[i]);
+                for (int64_t j = k0; j < k1; ++j) {
+                    float aj = fabsf(v[j]);
+                    if (aj > ai || (aj == ai && j < i)) ++rank;
+                }
+                int8_t s = v[i] > 0.0f ? 1 : (v[i] < 0.0f ? -1 : 0);
+                t[n * K + i] = rank < best_cnt ? s : 0;
+            }
+            volatile float alpha = best_cnt ? best_sum / (float)best_cnt : 0.0f;
+            scales[n * G + g] = oracle_float_to_half(alpha);
+        }
+    }
+    return ORACLE_OK;
 }
