@@ -109,18 +109,29 @@ typedef struct tern_matrix {
  * out: device, 16-byte aligned, tern_tiled_scales_bytes() bytes.
  */
 tern_status tern_tiled_scales_bytes(int32_t fmt, int32_t N, int32_t K, size_t *bytes);
+/* Errors (both): TERN_EINVAL for an unknown format, N or K < 1, a NULL or
+ * misaligned pointer; tern_retile_scales returns TERN_ECUDA when its launch
+ * fails. */
 tern_status tern_retile_scales(const tern_matrix *W, uint16_t *out, void *stream);
 
-/* Human-readable name of a status code (static storage). */
+/* Human-readable name of a status code (static storage).  Library plumbing:
+ * the pages have no counterpart. */
 const char *tern_status_string(tern_status s);
 
-/* Message of the last failure on the calling host thread ("" if none). */
+/* Message of the last failure on the calling host thread ("" if none).
+ * Library plumbing: the pages have no counterpart. */
 const char *tern_last_error(void);
 
 /*
  * Sizes of the device layout for an N x K matrix: the minimal row stride
  * (used row bytes rounded up to 16), the packed bytes N*row_stride and the
  * scale bytes 2*N*ceil(K/group).  Any output pointer may be NULL.
+ * The two densities are the pages': base-3 close to 1.6 bit per trit (Bonsai
+ * page, "后面还有没有优化空间"; a trit carries log2 3 = 1.585 bits, page
+ * pwwt.cn/news/5175886 section 1.1) and 2 bit per trit in a 2-bit field
+ * (same section; Bonsai page, "PQ2 会不会快很多"), plus one FP16 scale per
+ * group (4sapi page, section 三).  Errors: TERN_EINVAL for an unknown format
+ * or N, K, group < 1.
  */
 tern_status tern_packed_size(int32_t fmt, int32_t N, int32_t K, int32_t group,
                              int64_t *row_stride, size_t *packed_bytes,
@@ -128,11 +139,19 @@ tern_status tern_packed_size(int32_t fmt, int32_t N, int32_t K, int32_t group,
 
 /* Bytes per row of the canonical (file) encodings: base-3 = ceil(K/5)
  * (byte value sum_{i<5} t_i 3^i over K = 5j+i, least significant digit
- * first), 2-bit = ceil(K/4) (bits [2i,2i+1] of byte j hold K = 4j+i). */
+ * first), 2-bit = ceil(K/4) (bits [2i,2i+1] of byte j hold K = 4j+i).  These
+ * are the PTQ1_0-style (5 trits a byte) and PQ2-style (4 trits a byte) rows
+ * of the Bonsai page ("Decode 为什么只能算一般", "PQ2 会不会快很多"); the
+ * digit order is this library's reading, the pages give none.  Errors:
+ * TERN_EINVAL for an unknown format, K < 1 or a NULL `bytes`. */
 tern_status tern_canonical_row_bytes(int32_t fmt, int32_t K, int64_t *bytes);
 
 /*
- * Pack trits into the device layout.
+ * Pack trits into the device layout: the packing step that ends post-training
+ * ternarisation (page pwwt.cn/news/5175886, section 1.2: quantised weights
+ * and scales are packed in a fixed format), in the order the decode kernels
+ * consume the codes (Bonsai page, "后面还有没有优化空间": re-tile codes at
+ * load time into consumption order).
  *  trits: device int8 [N][K] in {-1, 0, +1}.
  *  packed_out: device, 16-byte aligned, N*row_stride bytes (row_stride as in
  *    tern_matrix).  Every byte of every row is written.
@@ -143,20 +162,26 @@ tern_status tern_pack(int32_t fmt, const int8_t *trits, int32_t N, int32_t K,
                       void *packed_out, int64_t row_stride, int32_t *d_invalid,
                       void *stream);
 
-/* Inverse of tern_pack: trits_out device int8 [N][K].  Invalid codes (D3
- * bytes that are no code, D2 fields equal to 3, padding digits other than
- * t = 1) are counted in d_invalid (may be NULL) and unpacked as 0. */
+/* Inverse of tern_pack: trits_out device int8 [N][K] -- the "unpack base-3,
+ * restore -1/0/+1" step of the Bonsai page ("Decode 为什么只能算一般"),
+ * written out to memory for tests.  Invalid codes (D3 bytes that are no
+ * code, D2 fields equal to 3, padding digits other than t = 1) are counted in
+ * d_invalid (may be NULL) and unpacked as 0.  Errors: TERN_EINVAL for a bad
+ * matrix or a NULL output. */
 tern_status tern_unpack(const tern_matrix *W, int8_t *trits_out,
                         int32_t *d_invalid, void *stream);
 
-/* Load-time re-tile: canonical bytes (device [N][canonical row bytes],
- * rows contiguous) into the device layout.  Invalid canonical codes are
- * counted in d_invalid (may be NULL). */
+/* Load-time re-tile (Bonsai page, "后面还有没有优化空间": rearrange the codes
+ * at load time in the order the integer dot product consumes them):
+ * canonical bytes (device [N][canonical row bytes], rows contiguous) into
+ * the device layout.  Invalid canonical codes are counted in d_invalid (may
+ * be NULL).  Errors: TERN_EINVAL for bad shapes, strides or pointers. */
 tern_status tern_import(int32_t fmt, const uint8_t *canonical, int32_t N,
                         int32_t K, void *packed_out, int64_t row_stride,
                         int32_t *d_invalid, void *stream);
 
-/* Device layout back to canonical bytes (device [N][canonical row bytes]). */
+/* Device layout back to canonical bytes (device [N][canonical row bytes]):
+ * the inverse of tern_import (same passage).  Errors as tern_unpack. */
 tern_status tern_export(const tern_matrix *W, uint8_t *canonical_out,
                         int32_t *d_invalid, void *stream);
 
@@ -183,10 +208,17 @@ tern_status act_quant_fwht(const void *x, int32_t x_is_fp16, int32_t M,
                            void *stream);
 
 /*
- * Ternary GEMV / skinny GEMM for decode, M = 1..16 token rows:
+ * Ternary GEMV / skinny GEMM for decode, M = 1..16 token rows (Bonsai page,
+ * "Decode 为什么只能算一般": batch-1 decode is a matrix-vector product that
+ * reads every packed weight once per token; the kernel unpacks the codes,
+ * restores -1/0/+1, reads the group scale and takes an integer dot product,
+ * never writing dequantised weights back; 4sapi page, section 三: add or
+ * subtract by sign, then multiply by the FP16 group scale):
  *   y[m][n] = residual[m][n] + s_x[m] * sum_g s_w[n][g] * P[m][n][g],
  *   P[m][n][g] = sum_{k in group g} w[n][k] * q[m][k]   (exact int32),
  * with residual taken as 0 when `residual` is NULL.
+ * Errors: TERN_EINVAL for a bad matrix, M outside 1..16, misaligned or NULL
+ * buffers or strides; TERN_ECUDA when the launch fails.
  *  q: device int8 [M][ldq], 16-byte aligned, ldq >= K, ldq % 16 == 0
  *     (bytes past K are ignored).  s_x: device fp32 [M].
  *  residual, y: device fp32 [M][ldy], ldy >= N; residual may equal y.
@@ -229,14 +261,19 @@ tern_status tern_gateup_swiglu(const tern_matrix *Wg, const tern_matrix *Wu,
 
 /*
  * Test hook: the exact integer group partials P[m][n][g] (device int32
- * [M][N][ceil(K/group)]) of the same kernels tern_gemv runs.
+ * [M][N][ceil(K/group)]) of the integer dot product of tern_gemv (Bonsai
+ * page, "Decode 为什么只能算一般": integer dot of the restored trits with the
+ * quantised activation), as the CUDA-core engine computes them.
  */
 tern_status tern_debug_group_partials(const tern_matrix *W, const int8_t *q,
                                       int32_t ldq, int32_t M, int32_t *P,
                                       void *stream);
 
 /*
- * Activation statistics, the input of the fused quantisation below.  For each
+ * Activation statistics, the input of the fused quantisation below (Bonsai
+ * page, "Decode 为什么只能算一般": activations are re-quantised between the
+ * matmuls of a layer, so a producer can hand its consumer the statistics
+ * that quantisation needs).  For each
  * token row m of x (fp32 [M][ldx], 16-byte aligned, ldx % 4 == 0) and each
  * 128-element block b of its first K elements (the last block zero-padded):
  *   stats[(m*stats_ld + b)*4 + 0] = max |x_b|
@@ -278,7 +315,9 @@ tern_status tern_gateup_swiglu_fused(const tern_matrix *Wg, const tern_matrix *W
 
 /*
  * Streamed forms of tern_gemv_fused / tern_gateup_swiglu_fused for decode
- * with M = 1 or 2 token rows, same results and arguments apart from these:
+ * with M = 1 or 2 token rows (Bonsai page, "Decode 为什么只能算一般": at batch
+ * 1 the memory controller spends decode moving weights, so each projection
+ * should cost about its bytes), same results and arguments apart from these:
  *  - the activation statistics are not needed: every CTA forms the row
  *    scale from x itself (max |x|, or max |H x| with TERN_QUANT_FWHT128);
  *  - W->scales_tiled must hold the re-tiled scales (tern_retile_scales);
@@ -289,7 +328,9 @@ tern_status tern_gateup_swiglu_fused(const tern_matrix *Wg, const tern_matrix *W
  *    what it wrote, so the workspace is all zero again after each call and
  *    one workspace, sized for the largest call, serves a whole chain of
  *    calls of any sizes on one stream (calls that may overlap need separate
- *    workspaces).
+ *    workspaces).  The exception is a call whose bounded wait ran out
+ *    (tern_device_error reports it): a partial published after the wait
+ *    gave up can stay behind, so zero the workspace again before reusing it.
  * One CTA per SM streams an equal share of the matrix's 32-row x 128-byte
  * tiles; with TERN_MATRIX_STATIC the tiles start streaming before the
  * previous kernel on the stream has finished.  x must not overlap y / h.
@@ -332,6 +373,46 @@ tern_status tern_gemv_streamed_noalloc(const tern_matrix *W, const float *x, int
                                        float *y, int32_t ldy, void *stream);
 
 /*
+ * Test hook of the streamed kernels (the integer dot product and the
+ * in-kernel quantisation of the Bonsai page, "Decode 为什么只能算一般"): runs
+ * tern_gemv_streamed (W1 == NULL, no residual) or tern_gateup_swiglu_streamed
+ * (W1 = up matrix) with the same arguments and the same kernel, instantiated
+ * to also write
+ *   q_out[m][k] (k < K, row stride ldq_out >= K): the int8 input codes, and
+ *   s_x_out[m]: the row scales, both as CTA 0 holds them after quantising;
+ *   P_out[((mat * M + m) * N + n) * G + g] (G = ceil(K/128), mat 0 = W0,
+ *   1 = W1): every exact int32 group partial sum_{k in g} w[n][k] q[m][k].
+ * Outputs are device buffers owned by the caller; errors as
+ * tern_gemv_streamed, and TERN_EINVAL when an output is missing.
+ */
+tern_status tern_debug_streamed(const tern_matrix *W0, const tern_matrix *W1, const float *x,
+                                int32_t ldx, int32_t qflags, int32_t M, float *out, int32_t ldo,
+                                int8_t *q_out, int32_t ldq_out, float *s_x_out, int32_t *P_out,
+                                void *workspace, size_t ws_bytes, void *stream);
+
+/*
+ * Test hook of the prefill GEMM (the tensor-core product of the Bonsai page,
+ * "Decode 为什么只能算一般": prefill is a large matrix multiply): tern_gemm
+ * with the same arguments and kernel, instantiated to also write every exact
+ * int32 group partial P[(m * N + n) * ceil(K/128) + g] as the tensor cores
+ * accumulated it.  P: device int32, caller-owned.  Errors as tern_gemm.
+ */
+tern_status tern_debug_gemm_partials(const tern_matrix *W, const int8_t *q, int32_t ldq,
+                                     const float *s_x, int32_t M, float *y, int32_t ldy, int32_t *P,
+                                     void *stream);
+
+/*
+ * Test hook of the bounded waits (no counterpart on the pages): one kernel
+ * waits on something nothing will ever complete -- kind 0: an mbarrier phase
+ * (the form of the weight-ring and cluster waits), kind 1: a tagged 64-bit
+ * word (the form of the wait for a neighbour's partial) -- for at most
+ * budget_cycles SM cycles (1 .. 2e8), then records the timeout in the
+ * device error word and returns.  tern_device_error then reports it.
+ * Errors: TERN_EINVAL for a bad kind or budget.
+ */
+tern_status tern_debug_bounded_wait(int32_t kind, int64_t budget_cycles, void *stream);
+
+/*
  * Test hook for the tensor-core path (no counterpart on the pages; it pins
  * the tcgen05 encodings the kernels use): one CTA computes
  *   D[m][n] = sum_k A[m][k] * B[n][k]   (int32, exact)
@@ -357,8 +438,11 @@ tern_status tern_debug_select_engine(int32_t engine);
 
 /*
  * Reads and clears the device error word of the current device: 0 when no
- * bounded wait in a kernel ran out since the last call, else a nonzero code.
- * Synchronises `stream`.
+ * bounded wait in a kernel ran out since the last call, else a nonzero code
+ * (1: a wait on an mbarrier, a cluster peer or a neighbour's partial ran
+ * out).  Synchronises `stream`.  Library plumbing (no counterpart on the
+ * pages).  After a nonzero code, zero every streamed workspace the failed
+ * calls used before using it again.
  */
 tern_status tern_device_error(int32_t *code_out, void *stream);
 

@@ -21,11 +21,12 @@ FLAGS = ARCH + ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC", "-rdc=t
 LIBS = {
     "libtern.so": ["csrc/tern_api.cu", "csrc/tern_format.cu", "csrc/tern_quant.cu",
                    "csrc/tern_gemv.cu", "csrc/tern_gemv_tc.cu", "csrc/tern_gemv_stream.cu",
-                   "csrc/tern_noalloc.cu", "csrc/tern_gemm.cu", "csrc/tern_tcdebug.cu"],
+                   "csrc/tern_noalloc.cu", "csrc/tern_gemm.cu", "csrc/tern_tcdebug.cu",
+                   "csrc/tern_debug.cu"],
     "libtern_synth.so": ["synth_csrc/tern_synth.cu"],
 }
 HEADERS = ["csrc/tern_common.cuh", "csrc/tern_internal.h", "csrc/tern_tc.cuh",
-           "csrc/tern_gemv_common.cuh"]
+           "csrc/tern_gemv_common.cuh", "csrc/tern_gemv_stream.cuh"]
 
 
 def _newest(paths):

@@ -323,10 +323,21 @@ tern_status tern_stream_workspace_bytes(int32_t fmt, int32_t N, int32_t M, int32
     return TERN_OK;
 }
 
-static tern_status run_streamed(const tern_matrix *W0, const tern_matrix *W1, const float *x,
+}  // extern "C"
+
+namespace tern {
+tern_status check_streamed_call(const tern_matrix *W0, const tern_matrix *W1, const float *x,
                                 int32_t ldx, int32_t qflags, int32_t M, const float *residual,
-                                float *out, int32_t ldo, void *workspace, size_t ws_bytes,
-                                void *stream, const char *name) {
+                                const float *out, int32_t ldo, const char *name) {
+    tern_status st = check_matrix(W0, name);
+    if (st != TERN_OK) return st;
+    if (W1) {
+        st = check_matrix(W1, name);
+        if (st != TERN_OK) return st;
+        if (W0->fmt != W1->fmt || W0->N != W1->N || W0->K != W1->K || W0->group != W1->group ||
+            W0->row_stride != W1->row_stride)
+            return fail(TERN_EINVAL, "%s: gate and up must share fmt, N, K, group, row_stride", name);
+    }
     if (M < 1 || M > 2) return fail(TERN_EUNSUPPORTED, "%s: the streamed kernels take M = 1 or 2", name);
     if (!W0->scales_tiled || (W1 && !W1->scales_tiled))
         return fail(TERN_EINVAL, "%s: scales_tiled is required (tern_retile_scales)", name);
@@ -337,6 +348,24 @@ static tern_status run_streamed(const tern_matrix *W0, const tern_matrix *W1, co
         return fail(TERN_EINVAL, "%s: the Hadamard rotation needs K %% 128 == 0", name);
     if (!out || !aligned(out, 4) || ldo < W0->N) return fail(TERN_EINVAL, "%s: bad output or its stride", name);
     if (residual && !aligned(residual, 4)) return fail(TERN_EINVAL, "%s: bad residual", name);
+    return TERN_OK;
+}
+}  // namespace tern
+
+namespace {
+struct StreamDebug {
+    int8_t *q;
+    int32_t ldq;
+    float *s_x;
+    int32_t *P;
+};
+
+tern_status run_streamed(const tern_matrix *W0, const tern_matrix *W1, const float *x, int32_t ldx,
+                         int32_t qflags, int32_t M, const float *residual, float *out, int32_t ldo,
+                         void *workspace, size_t ws_bytes, void *stream, const char *name,
+                         const StreamDebug *dbg = nullptr) {
+    tern_status st = tern::check_streamed_call(W0, W1, x, ldx, qflags, M, residual, out, ldo, name);
+    if (st != TERN_OK) return st;
     const size_t need = tern::stream_workspace_bytes(W0->fmt, W0->N, M, W1 ? 2 : 1);
     if (!workspace || !aligned(workspace, 16) || ws_bytes < need)
         return fail(TERN_EINVAL, "%s: workspace missing, misaligned or too small", name);
@@ -367,16 +396,25 @@ static tern_status run_streamed(const tern_matrix *W0, const tern_matrix *W1, co
     S.ws_bytes = ws_bytes;
     S.num_sms = sms;
     const char *why = nullptr;
-    e = tern::launch_gemv_stream(S, static_cast<cudaStream_t>(stream), &why);
+    if (dbg) {
+        S.dbg_q = dbg->q;
+        S.dbg_ldq = dbg->ldq;
+        S.dbg_sx = dbg->s_x;
+        S.dbg_P = dbg->P;
+        e = tern::launch_gemv_stream_debug(S, static_cast<cudaStream_t>(stream), &why);
+    } else {
+        e = tern::launch_gemv_stream(S, static_cast<cudaStream_t>(stream), &why);
+    }
     if (why) return fail(TERN_EUNSUPPORTED, "%s", why);
     return cuda_status(e, name);
 }
+}  // namespace
+
+extern "C" {
 
 tern_status tern_gemv_streamed(const tern_matrix *W, const float *x, int32_t ldx, int32_t qflags,
                                int32_t M, const float *residual, float *y, int32_t ldy,
                                void *workspace, size_t ws_bytes, void *stream) {
-    tern_status st = check_matrix(W, "tern_gemv_streamed");
-    if (st != TERN_OK) return st;
     return run_streamed(W, nullptr, x, ldx, qflags, M, residual, y, ldy, workspace, ws_bytes, stream,
                         "tern_gemv_streamed");
 }
@@ -385,19 +423,25 @@ tern_status tern_gateup_swiglu_streamed(const tern_matrix *Wg, const tern_matrix
                                         int32_t ldx, int32_t qflags, int32_t M, float *h,
                                         int32_t ldh, void *workspace, size_t ws_bytes,
                                         void *stream) {
-    tern_status st = check_matrix(Wg, "tern_gateup_swiglu_streamed (gate)");
-    if (st != TERN_OK) return st;
-    st = check_matrix(Wu, "tern_gateup_swiglu_streamed (up)");
-    if (st != TERN_OK) return st;
-    if (Wg->fmt != Wu->fmt || Wg->N != Wu->N || Wg->K != Wu->K || Wg->group != Wu->group ||
-        Wg->row_stride != Wu->row_stride)
-        return fail(TERN_EINVAL, "tern_gateup_swiglu_streamed: gate and up must share fmt, N, K, group, row_stride%s");
     return run_streamed(Wg, Wu, x, ldx, qflags, M, nullptr, h, ldh, workspace, ws_bytes, stream,
                         "tern_gateup_swiglu_streamed");
 }
 
-tern_status tern_gemm(const tern_matrix *W, const int8_t *q, int32_t ldq, const float *s_x,
-                      int32_t M, float *y, int32_t ldy, void *stream) {
+tern_status tern_debug_streamed(const tern_matrix *W0, const tern_matrix *W1, const float *x,
+                                int32_t ldx, int32_t qflags, int32_t M, float *out, int32_t ldo,
+                                int8_t *q_out, int32_t ldq_out, float *s_x_out, int32_t *P_out,
+                                void *workspace, size_t ws_bytes, void *stream) {
+    const char *name = "tern_debug_streamed";
+    if (!W0) return fail(TERN_EINVAL, "%s: null matrix", name);
+    if (!q_out || ldq_out < W0->K || !s_x_out || !aligned(s_x_out, 4) || !P_out || !aligned(P_out, 4))
+        return fail(TERN_EINVAL, "%s: q_out (ldq_out >= K), s_x_out and P_out are required", name);
+    const StreamDebug dbg = {q_out, ldq_out, s_x_out, P_out};
+    return run_streamed(W0, W1, x, ldx, qflags, M, nullptr, out, ldo, workspace, ws_bytes, stream, name,
+                        &dbg);
+}
+
+static tern_status run_gemm(const tern_matrix *W, const int8_t *q, int32_t ldq, const float *s_x,
+                            int32_t M, float *y, int32_t ldy, int32_t *dbg_P, void *stream) {
     tern_status st = check_matrix(W, "tern_gemm");
     if (st != TERN_OK) return st;
     if (M < 1) return fail(TERN_EINVAL, "tern_gemm: M must be >= 1%s");
@@ -419,10 +463,31 @@ tern_status tern_gemm(const tern_matrix *W, const int8_t *q, int32_t ldq, const 
     L.s_x = s_x;
     L.y = y;
     L.ldy = ldy;
+    L.dbg_P = dbg_P;
     const char *why = nullptr;
     cudaError_t e = tern::launch_gemm(L, static_cast<cudaStream_t>(stream), &why);
     if (why) return fail(TERN_EUNSUPPORTED, "tern_gemm: %s", why);
     return cuda_status(e, "tern_gemm");
+}
+
+tern_status tern_gemm(const tern_matrix *W, const int8_t *q, int32_t ldq, const float *s_x,
+                      int32_t M, float *y, int32_t ldy, void *stream) {
+    return run_gemm(W, q, ldq, s_x, M, y, ldy, nullptr, stream);
+}
+
+tern_status tern_debug_gemm_partials(const tern_matrix *W, const int8_t *q, int32_t ldq,
+                                     const float *s_x, int32_t M, float *y, int32_t ldy, int32_t *P,
+                                     void *stream) {
+    if (!P || !aligned(P, 4)) return fail(TERN_EINVAL, "tern_debug_gemm_partials: bad P%s");
+    return run_gemm(W, q, ldq, s_x, M, y, ldy, P, stream);
+}
+
+tern_status tern_debug_bounded_wait(int32_t kind, int64_t budget_cycles, void *stream) {
+    if (kind != 0 && kind != 1) return fail(TERN_EINVAL, "tern_debug_bounded_wait: kind must be 0 or 1%s");
+    if (budget_cycles < 1 || budget_cycles > 200000000LL)
+        return fail(TERN_EINVAL, "tern_debug_bounded_wait: budget must be 1 .. 2e8 cycles%s");
+    return cuda_status(tern::launch_debug_wait(kind, budget_cycles, static_cast<cudaStream_t>(stream)),
+                       "tern_debug_bounded_wait");
 }
 
 tern_status tern_debug_select_engine(int32_t engine) {

@@ -60,14 +60,15 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
     return ok != 0;
 }
 
-// Waits for phase `parity` of `bar` to complete, at most kWaitBudgetCycles.
+// Waits for phase `parity` of `bar` to complete, at most `budget` SM cycles.
 // Returns false (and records kErrTmaTimeout) when the budget runs out.
-__device__ __forceinline__ bool mbar_wait_bounded(uint64_t *bar, uint32_t parity) {
+__device__ __forceinline__ bool mbar_wait_bounded(uint64_t *bar, uint32_t parity,
+                                                  long long budget = kWaitBudgetCycles) {
     if (mbar_try_wait(bar, parity)) return true;
     long long start = clock64();
     while (!mbar_try_wait(bar, parity)) {
         __nanosleep(kWaitBackoffNs);  // leave the issue slots to warps with work
-        if (clock64() - start > kWaitBudgetCycles) {
+        if (clock64() - start > budget) {
             atomicExch(&g_device_error, kErrTmaTimeout);
             return false;
         }
@@ -198,6 +199,25 @@ __device__ __forceinline__ unsigned long long ld_relaxed_gpu_u64(const unsigned 
     unsigned long long v;
     asm volatile("ld.relaxed.gpu.global.b64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
     return v;
+}
+
+// Reads the 64-bit word at p once its tag (high half) is nonzero, waiting at
+// most `budget` SM cycles for another CTA to publish it.  When the budget
+// runs out it records kErrTmaTimeout and returns the word as it stands (tag
+// still 0).
+__device__ __forceinline__ unsigned long long wait_tagged_word(const unsigned long long *p,
+                                                               long long budget = kWaitBudgetCycles) {
+    unsigned long long w = ld_relaxed_gpu_u64(p);
+    if ((w >> 32) != 0) return w;
+    const long long start = clock64();
+    while (((w = ld_relaxed_gpu_u64(p)) >> 32) == 0) {
+        __nanosleep(kWaitBackoffNs);
+        if (clock64() - start > budget) {
+            atomicExch(&g_device_error, kErrTmaTimeout);
+            break;
+        }
+    }
+    return w;
 }
 
 // Waits (bounded, like mbar_wait_bounded) for a phase completed by other CTAs

@@ -8,26 +8,28 @@
 // over the same packed weights; 4sapi page, section 三: integer products of
 // the signs, then one FP16 scale per group of 128.)
 //
-// One CTA computes a 128-row (n) x 128-token (m) tile of Y over all of K:
+// One CTA computes a 128-row (n) x 256-token (m) tile of Y over all of K,
+// with 22 warps:
 //  * warp 0 (TMA): per 128-byte superblock of codes, the 128 x 128 B code
-//    tile; per group of 128 K, the 128 x 128 B activation tile -- both with
+//    tile; per group of 128 K, the 256 x 128 B activation tile -- both with
 //    128-byte swizzle, no multicast;
-//  * warps 2..9 (decode; a thread = one weight row, one 64-K half of each
-//    group): the row's 32 code words of the superblock into registers, then
-//    per group the signed int8 weights w = t - 1 into a 128 x 128 B tile in
-//    the 128-byte-swizzled K-major layout the MMA reads (trits never leave
-//    the SM);
-//  * warp 1 (MMA, one thread): per group four tcgen05.mma (K = 32 each), A =
-//    weights, B = activations, int32 accumulator in tensor memory -- four
-//    accumulator buffers of 128 columns (all 512), so the tensor cores run
-//    up to three groups ahead of the epilogue;
-//  * warps 10..17 (epilogue, two per tensor-memory lane quarter, 64 token
+//  * warp 1 (MMA, one thread): per group four tcgen05.mma (M = 128, N = 256,
+//    K = 32 each), A = decoded weights, B = activations, int32 accumulator in
+//    tensor memory -- two accumulator buffers of 256 columns (all 512), so
+//    the tensor cores run one group ahead of the epilogue;
+//  * warps 2..5 (decode; a thread = one weight row): the row's 32 code words
+//    of the superblock into registers, then per group the signed int8
+//    weights w = t - 1 into a 128 x 128 B tile in the 128-byte-swizzled
+//    K-major layout the MMA reads (trits never leave the SM), two tiles in
+//    flight;
+//  * warps 6..21 (epilogue, four per tensor-memory lane quarter, 64 token
 //    columns each): the tile's group scales into shared memory once, then
 //    per group tcgen05.ld of the int32 partials, int -> float (exact: the
 //    partials are below 2^15), acc += s_w[n][g] * P in fp32 registers (group
 //    order, as the definition reads); at the end Y = s_x[m] * acc.
 // The per-group scale is why the accumulator is drained every 128 K: the
-// tensor cores accumulate only the exact integer partial of one group.
+// tensor cores accumulate only the exact integer partial of one group.  The
+// test-hook instantiation (DBG) also writes every partial P[m][n][g].
 #include "tern_gemv_common.cuh"
 #include "tern_tc.cuh"
 
@@ -58,6 +60,7 @@ struct GemmParams {
     const float *s_x;        // [M]
     float *y;
     int ldy;
+    int32_t *dbg_P;  // DBG kernels only: P [M][N][G]
 };
 
 struct GemmSmem {
@@ -115,7 +118,7 @@ __device__ __forceinline__ void decode_half(const uint32_t (&words)[32], int gg,
     }
 }
 
-template <int FMT>
+template <int FMT, bool DBG>
 __global__ void __launch_bounds__(kGmThreads, 1)
     gemm_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_q,
                 const GemmParams p) {
@@ -298,6 +301,15 @@ __global__ void __launch_bounds__(kGmThreads, 1)
 #pragma unroll
                 for (int c = 0; c < 8; ++c)
                     acc[8 * h + c] = fmaf(s, __int2float_rn(static_cast<int>(v[c])), acc[8 * h + c]);
+                if constexpr (DBG) {
+                    // test hook: the exact partials of this group
+#pragma unroll
+                    for (int c = 0; c < 8; ++c) {
+                        const int m = m0 + c0 + 8 * h + c;
+                        if (m < p.M && n < p.N)
+                            p.dbg_P[(static_cast<int64_t>(m) * p.N + n) * G + g] = static_cast<int>(v[c]);
+                    }
+                }
             }
         }
         pdl_wait();  // s_x comes from the previous kernel
@@ -337,6 +349,7 @@ cudaError_t launch_gemm(const GemmLaunch &L, cudaStream_t s, const char **why) {
     p.s_x = L.s_x;
     p.y = L.y;
     p.ldy = L.ldy;
+    p.dbg_P = L.dbg_P;
     CUtensorMap tm_w, tm_q;
     if (!make_tmap_2d(&tm_w, L.packed, static_cast<uint64_t>(L.row_bytes), static_cast<uint64_t>(L.N),
                       static_cast<uint64_t>(L.row_stride), kGmTileN) ||
@@ -351,7 +364,10 @@ cudaError_t launch_gemm(const GemmLaunch &L, cudaStream_t s, const char **why) {
         return cudaErrorInvalidValue;
     }
     cudaError_t e;
-    auto kern = L.fmt == TERN_FMT_BASE3 ? gemm_kernel<TERN_FMT_BASE3> : gemm_kernel<TERN_FMT_2BIT>;
+    auto kern = L.dbg_P ? (L.fmt == TERN_FMT_BASE3 ? gemm_kernel<TERN_FMT_BASE3, true>
+                                                   : gemm_kernel<TERN_FMT_2BIT, true>)
+                        : (L.fmt == TERN_FMT_BASE3 ? gemm_kernel<TERN_FMT_BASE3, false>
+                                                   : gemm_kernel<TERN_FMT_2BIT, false>);
     e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
     if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg = {};

@@ -360,14 +360,13 @@ EncodeTiledFn encode_fn() {
     return fn;
 }
 
-constexpr int kMaxDevices = 64;
 constexpr int kTargetCtas = 3 * 148;
 
 template <int FMT, int MT, int MODE, int XIN>
 cudaError_t launch_cc(const GemvLaunch &Lh, cudaStream_t s, const char **why) {
     constexpr int NMAT = (MODE == kModeSwiglu) ? 2 : 1;
     constexpr int POS = Fmt<FMT>::kPos;
-    static int smem_set[kMaxDevices] = {0};
+    static DeviceOnce once;  // kernel attributes, set once per device
 
     GemvParams p;
     fill_params(p, Lh);
@@ -399,20 +398,20 @@ cudaError_t launch_cc(const GemvLaunch &Lh, cudaStream_t s, const char **why) {
         return cudaErrorInvalidValue;
     }
     int dev = 0;
-    cudaError_t e = cudaGetDevice(&dev);
+    cudaError_t e = current_device(&dev);
     if (e != cudaSuccess) return e;
-    if (dev >= 0 && dev < kMaxDevices && !smem_set[dev]) {
-        e = cudaFuncSetAttribute(gemv_cc_kernel<FMT, MT, MODE, XIN>,
-                                 cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
-        if (e != cudaSuccess) return e;
+    e = once.run(dev, []() {
+        cudaError_t r = cudaFuncSetAttribute(gemv_cc_kernel<FMT, MT, MODE, XIN>,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
+        if (r != cudaSuccess) return r;
         // The largest shared-memory split for every launch, so that a launch
         // waiting on its predecessor (programmatic launch) can share its SMs:
         // launches whose splits differ cannot, and the SM drains first.
-        e = cudaFuncSetAttribute(gemv_cc_kernel<FMT, MT, MODE, XIN>,
-                                 cudaFuncAttributePreferredSharedMemoryCarveout, cudaSharedmemCarveoutMaxShared);
-        if (e != cudaSuccess) return e;
-        smem_set[dev] = 1;
-    }
+        return cudaFuncSetAttribute(gemv_cc_kernel<FMT, MT, MODE, XIN>,
+                                    cudaFuncAttributePreferredSharedMemoryCarveout,
+                                    cudaSharedmemCarveoutMaxShared);
+    });
+    if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(p.nsplit, rowgroups, 1);
     cfg.blockDim = dim3(kThreads, 1, 1);

@@ -414,7 +414,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     gemv_epilogue<MT, NMAT, MODE, XIN>(part, sx, p, split, rg, tid);
 }
 
-constexpr int kMaxDevices = 64;
 constexpr int kTargetCtas = 3 * 148;
 
 template <int FMT, int MT, int MODE, int XIN>
@@ -422,7 +421,7 @@ cudaError_t launch_tc(const GemvLaunch &Lh, cudaStream_t s, const char **why) {
     constexpr int NMAT = (MODE == kModeSwiglu) ? 2 : 1;
     constexpr int POS = Fmt<FMT>::kPos;
     constexpr int NB = TcShape<FMT, MT>::NB;
-    static int smem_set[kMaxDevices] = {0};
+    static DeviceOnce once;  // kernel attribute, set once per device
 
     GemvParams p;
     fill_params(p, Lh);
@@ -461,14 +460,13 @@ cudaError_t launch_tc(const GemvLaunch &Lh, cudaStream_t s, const char **why) {
         return cudaErrorInvalidValue;
     }
     int dev = 0;
-    cudaError_t e = cudaGetDevice(&dev);
+    cudaError_t e = current_device(&dev);
     if (e != cudaSuccess) return e;
-    if (dev >= 0 && dev < kMaxDevices && !smem_set[dev]) {
-        e = cudaFuncSetAttribute(gemv_tc_kernel<FMT, MT, MODE, XIN>,
-                                 cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
-        if (e != cudaSuccess) return e;
-        smem_set[dev] = 1;
-    }
+    e = once.run(dev, []() {
+        return cudaFuncSetAttribute(gemv_tc_kernel<FMT, MT, MODE, XIN>,
+                                    cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
+    });
+    if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(p.nsplit, rowgroups, 1);
     cfg.blockDim = dim3(kThreads, 1, 1);

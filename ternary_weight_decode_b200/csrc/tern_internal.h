@@ -6,11 +6,46 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <atomic>
+#include <mutex>
+
 #include "../../include/tern.h"
 
 namespace tern {
 
 inline int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
+
+// One-time set-up of a launch site on each device (kernel attributes, launch
+// plans).  Safe when several host threads make their first call at once: the
+// first caller on a device runs `setup` under a lock, later callers see its
+// result through an acquire load without locking.  A set-up that fails is
+// tried again on the next call.  Use as a function-local static.
+class DeviceOnce {
+  public:
+    static constexpr int kMaxDevices = 64;
+    template <typename F>
+    cudaError_t run(int dev, F &&setup) {
+        if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+        if (done_[dev].load(std::memory_order_acquire)) return cudaSuccess;
+        std::lock_guard<std::mutex> lock(mu_);
+        if (done_[dev].load(std::memory_order_relaxed)) return cudaSuccess;
+        const cudaError_t e = setup();
+        if (e == cudaSuccess) done_[dev].store(1, std::memory_order_release);
+        return e;
+    }
+
+  private:
+    std::mutex mu_;
+    std::atomic<int> done_[kMaxDevices]{};
+};
+
+// The current device, checked against DeviceOnce's range.
+inline cudaError_t current_device(int *dev) {
+    cudaError_t e = cudaGetDevice(dev);
+    if (e != cudaSuccess) return e;
+    if (*dev < 0 || *dev >= DeviceOnce::kMaxDevices) return cudaErrorInvalidDevice;
+    return cudaSuccess;
+}
 
 inline int64_t device_row_bytes(int fmt, int64_t K) {
     if (fmt == TERN_FMT_BASE3) return 4 * ((K + 19) / 20);
@@ -94,14 +129,31 @@ struct StreamLaunch {
     void *workspace;
     size_t ws_bytes;
     int num_sms;
+    // test hook only (launch_gemv_stream_debug): the int8 input codes [M][dbg_ldq]
+    // and row scales [M] as CTA 0 holds them, and every exact int32 group
+    // partial [NMAT][M][N][ceil(K/128)]
+    int8_t *dbg_q;
+    int dbg_ldq;
+    float *dbg_sx;
+    int32_t *dbg_P;
 };
 size_t stream_workspace_bytes(int fmt, int N, int M, int nmat);
 cudaError_t launch_gemv_stream(const StreamLaunch &S, cudaStream_t s, const char **why);
+// The same kernels instantiated with the test-hook outputs (S.dbg_*).
+cudaError_t launch_gemv_stream_debug(const StreamLaunch &S, cudaStream_t s, const char **why);
+// Host-side checks of a streamed call, everything but the workspace (W1 is
+// the up matrix of the SwiGLU form, else NULL).  Sets tern_last_error().
+tern_status check_streamed_call(const tern_matrix *W0, const tern_matrix *W1, const float *x,
+                                int32_t ldx, int32_t qflags, int32_t M, const float *residual,
+                                const float *out, int32_t ldo, const char *name);
 cudaError_t launch_gemv_tc(const GemvLaunch &L, cudaStream_t s, const char **why);
 void select_engine(int engine);  // 0: tensor cores, 1: CUDA cores (default)
 cudaError_t launch_act_stats(const float *x, int M, int K, int ldx, float *stats, int ld,
                              cudaStream_t s);
 cudaError_t read_clear_device_error(int *value, cudaStream_t s);
+// Test hook: one bounded wait that nothing satisfies (kind 0: an mbarrier
+// phase, kind 1: a tagged global word), with the given budget in SM cycles.
+cudaError_t launch_debug_wait(int kind, long long budget_cycles, cudaStream_t s);
 
 // 3-D view (byte in superblock, row, superblock) of a packed matrix's whole
 // superblocks: one box = box_sb consecutive superblocks of 32 rows.
@@ -123,6 +175,7 @@ struct GemmLaunch {
     const float *s_x;
     float *y;
     int ldy;
+    int32_t *dbg_P;  // test hook only: exact int32 group partials [M][N][ceil(K/128)]
 };
 cudaError_t launch_gemm(const GemmLaunch &L, cudaStream_t s, const char **why);
 

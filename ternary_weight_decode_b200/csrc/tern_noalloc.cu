@@ -45,10 +45,11 @@ cudaError_t scratch_address(void **out) {
 tern_status tern_gemv_streamed_noalloc(const tern_matrix *W, const float *x, int32_t ldx,
                                        int32_t qflags, int32_t M, const float *residual,
                                        float *y, int32_t ldy, void *stream) {
-    // A missing matrix, N < 1 or M outside 1..2 gets the streamed entry
-    // point's own message (it fails before it looks at the workspace).
-    if (!W || W->N < 1 || M < 1 || M > 2)
-        return tern_gemv_streamed(W, x, ldx, qflags, M, residual, y, ldy, nullptr, 0, stream);
+    // Every host-side check of the streamed entry point first, so that a
+    // call that is rejected leaves the shared array untouched.
+    const tern_status st = tern::check_streamed_call(W, nullptr, x, ldx, qflags, M, residual, y, ldy,
+                                                     "tern_gemv_streamed_noalloc");
+    if (st != TERN_OK) return st;
     const size_t bytes = TERN_NOALLOC_SCRATCH_BYTES;
     const size_t need = tern::stream_workspace_bytes(W->fmt, W->N, M, 1);
     if (need > bytes) {

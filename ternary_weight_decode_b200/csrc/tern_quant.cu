@@ -142,26 +142,24 @@ cudaError_t launch_act_quant(const void *x, bool fp16, int M, int K, int ldx, in
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    cudaError_t e;
-    if (fp16) {
-        static bool init = false;
-        if (!init) {
-            e = cudaFuncSetAttribute(act_quant_kernel<true>,
-                                     cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
-            if (e != cudaSuccess) return e;
-            init = true;
-        }
+    // The shared-memory limit is a property of the kernel on each device:
+    // set once per device (thread-safe), for both input types.
+    static DeviceOnce once;
+    int dev = 0;
+    cudaError_t e = current_device(&dev);
+    if (e != cudaSuccess) return e;
+    e = once.run(dev, []() {
+        cudaError_t r = cudaFuncSetAttribute(act_quant_kernel<true>,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
+        if (r != cudaSuccess) return r;
+        return cudaFuncSetAttribute(act_quant_kernel<false>,
+                                    cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
+    });
+    if (e != cudaSuccess) return e;
+    if (fp16)
         e = cudaLaunchKernelEx(&cfg, act_quant_kernel<true>, x, K, ldx, fwht_block, rmsnorm, q, ldq, s_x);
-    } else {
-        static bool init = false;
-        if (!init) {
-            e = cudaFuncSetAttribute(act_quant_kernel<false>,
-                                     cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
-            if (e != cudaSuccess) return e;
-            init = true;
-        }
+    else
         e = cudaLaunchKernelEx(&cfg, act_quant_kernel<false>, x, K, ldx, fwht_block, rmsnorm, q, ldq, s_x);
-    }
     if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }

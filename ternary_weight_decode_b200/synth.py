@@ -76,13 +76,34 @@ def hash_at(seed: int, stream: int, idx: np.ndarray) -> np.ndarray:
 
 
 def trits_rows(seed: int, stream: int, rows: np.ndarray, K: int) -> np.ndarray:
-    """Trits int8 [len(rows), K] of the matrix (seed, stream) at the given rows."""
-    rows = np.asarray(rows, dtype=np.uint64).reshape(-1, 1)
-    idx = rows * np.uint64(K) + np.arange(K, dtype=np.uint64).reshape(1, -1)
-    u = hash_at(seed, stream, idx) >> np.uint64(32)
-    out = np.zeros(u.shape, dtype=np.int8)
-    out[u < np.uint64(T_NEG)] = -1
-    out[u >= np.uint64(T_POS)] = 1
+    """Trits int8 [len(rows), K] of the matrix (seed, stream) at the given rows:
+    h(seed, stream, row * K + col) as hash_at defines it, evaluated a few rows
+    at a time with in-place numpy steps (the same bits, without full-size
+    temporaries)."""
+    rows = np.asarray(rows, dtype=np.uint64).ravel()
+    out = np.empty((rows.size, K), np.int8)
+    key = np.uint64(stream_key(seed, stream))
+    col1 = np.arange(1, K + 1, dtype=np.uint64).reshape(1, -1)  # idx + 1
+    chunk = max(1, (1 << 18) // max(K, 1))
+    c1, c2 = np.uint64(0xBF58476D1CE4E5B9), np.uint64(0x94D049BB133111EB)
+    tn, tp = np.uint64(T_NEG), np.uint64(T_POS)
+    with np.errstate(over="ignore"):
+        for r0 in range(0, rows.size, chunk):
+            z = rows[r0:r0 + chunk].reshape(-1, 1) * np.uint64(K) + col1
+            z *= np.uint64(GAMMA)
+            z += key
+            t = z >> np.uint64(30)
+            z ^= t
+            z *= c1
+            np.right_shift(z, np.uint64(27), out=t)
+            z ^= t
+            z *= c2
+            np.right_shift(z, np.uint64(31), out=t)
+            z ^= t
+            z >>= np.uint64(32)
+            o = out[r0:r0 + chunk]
+            np.greater_equal(z, tp, out=o, casting="unsafe")  # +1
+            o -= (z < tn)                                        # -1
     return out
 
 

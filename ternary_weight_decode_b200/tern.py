@@ -89,6 +89,10 @@ def lib() -> ctypes.CDLL:
                                                                p]),
                 "tern_gemv_streamed_noalloc": (ctypes.c_int, [pm, p, i32, i32, i32, p, p, i32, p]),
                 "tern_gemm": (ctypes.c_int, [pm, p, i32, p, i32, p, i32, p]),
+                "tern_debug_streamed": (ctypes.c_int, [pm, pm, p, i32, i32, i32, p, i32, p, i32, p, p,
+                                                       p, sz, p]),
+                "tern_debug_gemm_partials": (ctypes.c_int, [pm, p, i32, p, i32, p, i32, p, p]),
+                "tern_debug_bounded_wait": (ctypes.c_int, [i32, i64, p]),
                 "tern_gemv_fused": (ctypes.c_int, [pm, p, i32, p, i32, i32, i32, p, p, i32, p, i32, p]),
                 "tern_gateup_swiglu_fused": (ctypes.c_int, [pm, pm, p, i32, p, i32, i32, i32, p, i32,
                                                             p, i32, p]),
@@ -377,6 +381,43 @@ def tern_gateup_swiglu_streamed(Wg: TernMatrix, Wu: TernMatrix, x: torch.Tensor,
                                              _ptr(workspace),
                                              workspace.numel() * workspace.element_size(),
                                              _stream(stream)), "tern_gateup_swiglu_streamed")
+
+
+def tern_debug_streamed(W0: TernMatrix, W1: TernMatrix | None, x: torch.Tensor, out: torch.Tensor,
+                        q_out: torch.Tensor, s_x_out: torch.Tensor, P_out: torch.Tensor,
+                        workspace: torch.Tensor, qflags: int = 0, M: int | None = None, stream=None):
+    """Test hook: the streamed kernel (GEMV, or SwiGLU when W1 is given) also
+    writes its int8 input q_out [M, >=K], row scales s_x_out [M] and exact
+    group partials P_out int32 [NMAT, M, N, G]."""
+    M = x.shape[0] if M is None else M
+    assert x.dtype == torch.float32 and x.stride(1) == 1 and out.dtype == torch.float32
+    assert q_out.dtype == torch.int8 and s_x_out.dtype == torch.float32
+    assert P_out.dtype == torch.int32 and P_out.is_contiguous()
+    s0 = W0.struct()
+    s1 = None if W1 is None else ctypes.byref(W1.struct())
+    _check(lib().tern_debug_streamed(ctypes.byref(s0), s1, _ptr(x), x.stride(0), qflags, M, _ptr(out),
+                                     out.stride(0), _ptr(q_out), q_out.stride(0), _ptr(s_x_out),
+                                     _ptr(P_out), _ptr(workspace),
+                                     workspace.numel() * workspace.element_size(), _stream(stream)),
+           "tern_debug_streamed")
+
+
+def tern_debug_gemm_partials(W: TernMatrix, q: torch.Tensor, s_x: torch.Tensor, y: torch.Tensor,
+                             P: torch.Tensor, M: int | None = None, stream=None):
+    """Test hook: tern_gemm that also writes its exact group partials P int32 [M, N, G]."""
+    M = q.shape[0] if M is None else M
+    assert q.dtype == torch.int8 and q.stride(1) == 1 and y.dtype == torch.float32
+    assert P.dtype == torch.int32 and P.is_contiguous()
+    s = W.struct()
+    _check(lib().tern_debug_gemm_partials(ctypes.byref(s), _ptr(q), q.stride(0), _ptr(s_x), M, _ptr(y),
+                                          y.stride(0), _ptr(P), _stream(stream)),
+           "tern_debug_gemm_partials")
+
+
+def tern_debug_bounded_wait(kind: int, budget_cycles: int, stream=None):
+    """Test hook: a kernel whose bounded wait (0: mbarrier, 1: tagged word) runs out."""
+    _check(lib().tern_debug_bounded_wait(kind, budget_cycles, _stream(stream)),
+           "tern_debug_bounded_wait")
 
 
 ENGINE_TENSOR_CORES, ENGINE_CUDA_CORES = 0, 1

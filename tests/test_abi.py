@@ -130,3 +130,35 @@ def test_gemm_rejects_bad_arguments(ldq, M, ldy, q, y):
                        ctypes.c_void_p(y) if y else None, ldy, None)
     assert st == 1, lib.tern_last_error()
     assert b"tern_gemm" in lib.tern_last_error()
+
+
+@pytest.mark.parametrize("kind,budget", [(2, 1000), (-1, 1000), (0, 0), (1, 200000001)])
+def test_bounded_wait_hook_rejects_bad_arguments(kind, budget):
+    """Host validation only: no kernel is launched."""
+    lib = _lib()
+    assert lib.tern_debug_bounded_wait(kind, budget, None) == 1
+    assert b"tern_debug_bounded_wait" in lib.tern_last_error()
+
+
+def test_debug_streamed_requires_its_outputs():
+    lib = _lib()
+    m = _matrix(scales_tiled=16384)
+    st = lib.tern_debug_streamed(ctypes.byref(m), None, ctypes.c_void_p(4096), 256, 0, 1,
+                                 ctypes.c_void_p(4096), 4, None, 256, ctypes.c_void_p(4096),
+                                 ctypes.c_void_p(4096), ctypes.c_void_p(4096), 1 << 20, None)
+    assert st == 1 and b"q_out" in lib.tern_last_error()
+
+
+def test_noalloc_validates_before_touching_its_array():
+    """A call rejected on its arguments fails before any CUDA call (no GPU is
+    needed to see the error), so it cannot have cleared the shared array."""
+    lib = _lib()
+    m = _matrix(scales_tiled=16384)
+    # x misaligned
+    st = lib.tern_gemv_streamed_noalloc(ctypes.byref(m), ctypes.c_void_p(4100), 256, 0, 1, None,
+                                        ctypes.c_void_p(4096), 4, None)
+    assert st == 1 and b"x must be" in lib.tern_last_error()
+    # unknown qflags
+    st = lib.tern_gemv_streamed_noalloc(ctypes.byref(m), ctypes.c_void_p(4096), 256, 8, 1, None,
+                                        ctypes.c_void_p(4096), 4, None)
+    assert st == 1 and b"qflags" in lib.tern_last_error()

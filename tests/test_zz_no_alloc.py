@@ -35,6 +35,9 @@ def _input(seed, M, K):
 @pytest.mark.parametrize("N,K,M,qflags", [(5120, 5120, 1, RMS), (4100, 17408, 2, ROT),
                                           (37, 300, 1, 0), (7168, 5120, 2, RMS | ROT)])
 def test_noalloc_matches_streamed_on_two_calls(fmt, N, K, M, qflags):
+    """Same kernel, same fixed summation order: the results are identical
+    bit for bit to tern_gemv_streamed's, and within the oracle's tolerance."""
+    import oracle
     from gpu_util import make_matrix, tolerance
     w = synth.trits(77, 0, N, K)
     sw = synth.scales(77, 1, N, synth.groups(K))
@@ -51,9 +54,39 @@ def test_noalloc_matches_streamed_on_two_calls(fmt, N, K, M, qflags):
         tern.tern_gemv_streamed(W, x, y_ref, ws, qflags=qflags, residual=residual, M=M)
         tern.tern_gemv_streamed_noalloc(W, x, y, qflags=qflags, residual=residual, M=M)
         torch.cuda.synchronize()
-        ref = y_ref.cpu().numpy()
-        got = y.cpu().numpy()
-        assert np.max(np.abs(got - ref)) <= tolerance(ref), f"call {call}"
+        np.testing.assert_array_equal(y.cpu().numpy(), y_ref.cpu().numpy(), err_msg=f"call {call}")
+        if call == 0:
+            xh = x.cpu().numpy()[:, :K]
+            q, s = oracle.act_quant(xh, fwht_block=128 if qflags & ROT else 0,
+                                    rmsnorm=bool(qflags & RMS))
+            ref = oracle.gemv(w, sw, q, s)
+            assert np.max(np.abs(y.cpu().numpy() - ref)) <= tolerance(ref)
+    assert tern.tern_device_error() == 0
+
+
+@pytest.mark.gpu
+def test_noalloc_shared_array_large_then_small_and_mixed():
+    """Calls share one array: a large call (N = 129024 at M = 1, the whole
+    array) leaves its words cleared, and smaller calls of the other format
+    and of M = 2 that follow on the same array still give the workspace
+    path's results bit for bit."""
+    from gpu_util import make_matrix
+    seq = [(tern.TERN_FMT_BASE3, 129024, 640, 1), (tern.TERN_FMT_2BIT, 300, 1280, 2),
+           (tern.TERN_FMT_BASE3, 5120, 5120, 2), (tern.TERN_FMT_2BIT, 65024, 512, 2),
+           (tern.TERN_FMT_BASE3, 33, 20, 1), (tern.TERN_FMT_2BIT, 7168, 5120, 1)]
+    for i, (fmt, N, K, M) in enumerate(seq):
+        w = synth.trits(78, i, N, K)
+        sw = synth.scales(78, 100 + i, N, synth.groups(K))
+        W = make_matrix(fmt, w, sw).retile_scales()
+        x = _input(520 + 3 * i, M, K)
+        ws = tern.stream_workspace(fmt, N, M, False)
+        y_ref = torch.zeros((M, N), dtype=torch.float32, device="cuda")
+        y = torch.ones((M, N), dtype=torch.float32, device="cuda")
+        tern.tern_gemv_streamed(W, x, y_ref, ws, qflags=RMS, M=M)
+        tern.tern_gemv_streamed_noalloc(W, x, y, qflags=RMS, M=M)
+        torch.cuda.synchronize()
+        np.testing.assert_array_equal(y.cpu().numpy(), y_ref.cpu().numpy(), err_msg=f"call {i}")
+        del W, x, ws, y, y_ref
     assert tern.tern_device_error() == 0
 
 
