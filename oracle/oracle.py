@@ -25,6 +25,7 @@ _lib = None
 
 FMT_BASE3 = 0
 FMT_2BIT = 1
+FMT_BITPLANE = 2
 
 
 class OracleError(ValueError):
@@ -52,7 +53,8 @@ def _load():
             p = ctypes.c_void_p
             lib.oracle_half_to_double.restype = ctypes.c_double
             lib.oracle_half_to_double.argtypes = [ctypes.c_uint16]
-            for name in ("oracle_base3_row_bytes", "oracle_2bit_row_bytes"):
+            for name in ("oracle_base3_row_bytes", "oracle_2bit_row_bytes",
+                         "oracle_bitplane_row_bytes"):
                 getattr(lib, name).restype = i64
                 getattr(lib, name).argtypes = [i64]
             lib.oracle_device_row_bytes.restype = i64
@@ -60,7 +62,7 @@ def _load():
             lib.oracle_groups.restype = i64
             lib.oracle_groups.argtypes = [i64, i64]
             for name in ("oracle_pack_base3", "oracle_unpack_base3", "oracle_pack_2bit",
-                         "oracle_unpack_2bit"):
+                         "oracle_unpack_2bit", "oracle_pack_bitplane", "oracle_unpack_bitplane"):
                 getattr(lib, name).restype = i32
                 getattr(lib, name).argtypes = [p, i64, i64, p]
             for name in ("oracle_pack_device", "oracle_unpack_device"):
@@ -165,6 +167,27 @@ def unpack_2bit(b: np.ndarray, K: int) -> np.ndarray:
     N = b.shape[0]
     w = np.zeros((N, K), np.int8)
     _check(_load().oracle_unpack_2bit(_ptr(b), N, K, _ptr(w)), "unpack_2bit")
+    return w
+
+
+def bitplane_row_bytes(K: int) -> int:
+    return int(_load().oracle_bitplane_row_bytes(K))
+
+
+def pack_bitplane(w: np.ndarray) -> np.ndarray:
+    """Canonical bit planes [N, 2 * ceil(K/8)]: the nonzero plane, then the sign plane."""
+    w = _c(w, np.int8)
+    N, K = w.shape
+    out = np.zeros((N, bitplane_row_bytes(K)), np.uint8)
+    _check(_load().oracle_pack_bitplane(_ptr(w), N, K, _ptr(out)), "pack_bitplane")
+    return out
+
+
+def unpack_bitplane(b: np.ndarray, K: int) -> np.ndarray:
+    b = _c(b, np.uint8)
+    N = b.shape[0]
+    w = np.zeros((N, K), np.int8)
+    _check(_load().oracle_unpack_bitplane(_ptr(b), N, K, _ptr(w)), "unpack_bitplane")
     return w
 
 

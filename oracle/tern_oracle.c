@@ -46,6 +46,12 @@
  *  R9 decode chain glue (the pages give no norm or attention detail): a
  *     weightless RMSNorm of the unrotated row folded into the scale only,
  *     s_x / sqrt(mean(x^2) + 1e-6), which leaves every int8 code unchanged.
+ *  R11 bit-plane format (Bonsai page, "后面还有没有优化空间", first direction:
+ *     split the weights into a "nonzero" and a "sign" bit plane, about 2 bits
+ *     per weight, for a cheaper decode): n = (w != 0), s = (w < 0).
+ *     Canonical row: ceil(K/8) bytes of the n plane, then ceil(K/8) bytes of
+ *     the s plane, bit k mod 8 of byte k/8; bits past K are 0; an s bit set
+ *     where n is 0 is invalid (error 1).
  *  R10 ternarisation (pwwt.cn/news/5175886, section 1.2: per block, two
  *     thresholds -- values between them become 0, the two sides +1 / -1 --
  *     and a scale chosen to make the residual small; m.nxbn.cn/news/172464,
@@ -69,8 +75,12 @@
  *     (digit i = 0 most significant).  Row bytes used: 4*ceil(K/20).
  *  D2 (2-bit): a 4-byte word w covers K in [16w, 16w+16).  Bits [2i, 2i+1]
  *     of byte j hold t for K = 16w + 4i + j.  Row bytes used: 4*ceil(K/16).
- *  Both: positions past K hold t = 1; bytes past the used row bytes up to the
- *  row stride are 0.
+ *  DB (bit-plane): 4-byte words in pairs; pair p of a row covers K in
+ *     [32p, 32p+32): word 2p is the n plane, word 2p+1 the s plane, and bit
+ *     8j + i of each holds K = 32p + 4i + j (i = 0..7, j = 0..3).  Row bytes
+ *     used: 8*ceil(K/32).
+ *  D3, D2: positions past K hold t = 1; DB: positions past K hold n = s = 0
+ *  (w = 0).  Bytes past the used row bytes up to the row stride are 0.
  */
 #include <math.h>
 #include <stdint.h>
@@ -183,11 +193,46 @@ int oracle_unpack_2bit(const uint8_t *b, int64_t N, int64_t K, int8_t *w) {
     return ORACLE_OK;
 }
 
+/* Canonical bit-plane: the n plane then the s plane, 1 bit per weight (R11). */
+int64_t oracle_bitplane_row_bytes(int64_t K) { return 2 * ((K + 7) / 8); }
+
+int oracle_pack_bitplane(const int8_t *w, int64_t N, int64_t K, uint8_t *out) {
+    int64_t P = (K + 7) / 8, B = 2 * P;
+    for (int64_t n = 0; n < N; ++n) {
+        memset(out + n * B, 0, (size_t)B);
+        for (int64_t k = 0; k < K; ++k) {
+            int v = w[n * K + k];
+            if (v < -1 || v > 1) return ORACLE_EINVAL;
+            if (v != 0) out[n * B + k / 8] |= (uint8_t)(1u << (k % 8));
+            if (v < 0) out[n * B + P + k / 8] |= (uint8_t)(1u << (k % 8));
+        }
+    }
+    return ORACLE_OK;
+}
+
+int oracle_unpack_bitplane(const uint8_t *b, int64_t N, int64_t K, int8_t *w) {
+    int64_t P = (K + 7) / 8, B = 2 * P;
+    for (int64_t n = 0; n < N; ++n) {
+        for (int64_t k = 0; k < 8 * P; ++k) {
+            int nz = (b[n * B + k / 8] >> (k % 8)) & 1;
+            int sg = (b[n * B + P + k / 8] >> (k % 8)) & 1;
+            if (sg && !nz) return ORACLE_EINVAL;
+            if (k < K)
+                w[n * K + k] = (int8_t)(nz ? (sg ? -1 : 1) : 0);
+            else if (nz)
+                return ORACLE_EINVAL;
+        }
+    }
+    return ORACLE_OK;
+}
+
 /* ------------------------------------------------------------------ */
-/* Device layouts D3 / D2 (see the header comment). fmt 0 = D3, 1 = D2.   */
+/* Device layouts D3 / D2 / DB (see the header comment). fmt 0 = D3,
+ * 1 = D2, 2 = DB.                                                         */
 int64_t oracle_device_row_bytes(int fmt, int64_t K) {
     if (fmt == 0) return 4 * ((K + 19) / 20);
     if (fmt == 1) return 4 * ((K + 15) / 16);
+    if (fmt == 2) return 8 * ((K + 31) / 32);
     return -1;
 }
 
@@ -210,6 +255,18 @@ int oracle_pack_device(int fmt, const int8_t *w, int64_t N, int64_t K,
     for (int64_t n = 0; n < N; ++n) {
         uint8_t *row = out + n * row_stride;
         memset(row, 0, (size_t)row_stride);
+        if (fmt == 2) {
+            for (int64_t k = 0; k < K; ++k) {
+                int v = w[n * K + k];
+                if (v < -1 || v > 1) return ORACLE_EINVAL;
+                int64_t p = k / 32;
+                int i = (int)((k % 32) / 4), j = (int)(k % 4);
+                int bit = 8 * j + i;
+                if (v != 0) row[8 * p + bit / 8] |= (uint8_t)(1u << (bit % 8));
+                if (v < 0) row[8 * p + 4 + bit / 8] |= (uint8_t)(1u << (bit % 8));
+            }
+            continue;
+        }
         for (int64_t wd = 0; wd < used / 4; ++wd) {
             for (int j = 0; j < 4; ++j) {
                 int code = 0;
@@ -249,6 +306,21 @@ int oracle_unpack_device(int fmt, const uint8_t *b, int64_t N, int64_t K,
     if (used < 0 || row_stride < used) return ORACLE_EINVAL;
     for (int64_t n = 0; n < N; ++n) {
         const uint8_t *row = b + n * row_stride;
+        if (fmt == 2) {
+            for (int64_t k = 0; k < used * 4; ++k) { /* 32 positions per 8 bytes */
+                int64_t p = k / 32;
+                int i = (int)((k % 32) / 4), j = (int)(k % 4);
+                int bit = 8 * j + i;
+                int nz = (row[8 * p + bit / 8] >> (bit % 8)) & 1;
+                int sg = (row[8 * p + 4 + bit / 8] >> (bit % 8)) & 1;
+                if (sg && !nz) return ORACLE_EINVAL;
+                if (k < K)
+                    w[n * K + k] = (int8_t)(nz ? (sg ? -1 : 1) : 0);
+                else if (nz)
+                    return ORACLE_EINVAL;
+            }
+            continue;
+        }
         for (int64_t wd = 0; wd < used / 4; ++wd) {
             for (int j = 0; j < 4; ++j) {
                 int code = row[4 * wd + j];
