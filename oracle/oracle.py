@@ -90,6 +90,12 @@ def _load():
             lib.oracle_float_to_half.argtypes = [ctypes.c_float]
             lib.oracle_ternarize.restype = i32
             lib.oracle_ternarize.argtypes = [p, i64, i64, i64, i64, p, p]
+            lib.oracle_q4_0_quantize.restype = i32
+            lib.oracle_q4_0_quantize.argtypes = [p, i64, p, p]
+            lib.oracle_q4_0_dequantize.restype = None
+            lib.oracle_q4_0_dequantize.argtypes = [p, p, i64, p]
+            lib.oracle_attention_decode.restype = i32
+            lib.oracle_attention_decode.argtypes = [p, p, p, p, p, i64, i64, i64, i64, p]
             _lib = lib
     return _lib
 
@@ -312,3 +318,38 @@ def ternarize(w: np.ndarray, group: int = 128):
     sc = np.zeros((N, G), np.uint16)
     _check(_load().oracle_ternarize(_ptr(w), N, K, K, group, _ptr(t), _ptr(sc)), "ternarize")
     return t, sc.view(np.float16)
+
+
+# ---------------------------------------------------------------- Q4_0 KV attention
+def q4_0_quantize(x: np.ndarray):
+    """(d float16 [..., n/32], qs uint8 [..., n/32, 16]) of fp32 x [..., n], n % 32 == 0."""
+    x = _c(x, np.float32)
+    n = x.size
+    d = np.zeros(n // 32, np.uint16)
+    qs = np.zeros((n // 32, 16), np.uint8)
+    _check(_load().oracle_q4_0_quantize(_ptr(x), n, _ptr(d), _ptr(qs)), "q4_0_quantize")
+    lead = x.shape[:-1] + (x.shape[-1] // 32,)
+    return d.view(np.float16).reshape(lead), qs.reshape(lead + (16,))
+
+
+def q4_0_dequantize(d: np.ndarray, qs: np.ndarray) -> np.ndarray:
+    d = _c(np.asarray(d, np.float16).view(np.uint16), np.uint16)
+    qs = _c(qs, np.uint8)
+    n = d.size * 32
+    out = np.zeros(n, np.float64)
+    _load().oracle_q4_0_dequantize(_ptr(d), _ptr(qs), n, _ptr(out))
+    return out.reshape(d.shape[:-1] + (d.shape[-1] * 32,))
+
+
+def attention_decode(q, kd, kq, vd, vq):
+    """out fp64 [Hq, D] for q fp32 [Hq, D] and a Q4_0 cache: kd/vd float16
+    [Hkv, L, D/32], kq/vq uint8 [Hkv, L, D/32, 16]."""
+    q = _c(q, np.float32)
+    Hq, D = q.shape
+    Hkv, L = kd.shape[0], kd.shape[1]
+    args = [_c(np.asarray(a, np.float16).view(np.uint16), np.uint16) if i % 2 == 0 else _c(a, np.uint8)
+            for i, a in enumerate((kd, kq, vd, vq))]
+    out = np.zeros((Hq, D), np.float64)
+    _check(_load().oracle_attention_decode(_ptr(q), *[_ptr(a) for a in args], L, Hkv, Hq, D,
+                                          _ptr(out)), "attention_decode")
+    return out

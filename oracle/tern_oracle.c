@@ -52,6 +52,19 @@
  *     Canonical row: ceil(K/8) bytes of the n plane, then ceil(K/8) bytes of
  *     the s plane, bit k mod 8 of byte k/8; bits past K are 0; an s bit set
  *     where n is 0 is invalid (error 1).
+ *  R12 decode attention over a Q4_0 KV cache (Bonsai page, "先交代机器和配置":
+ *     K and V cached as Q4_0, Flash Attention on; the passage before "PQ2 会不会
+ *     快很多": the Q4 data is decoded inside attention).  Q4_0 is the block
+ *     format of the llama.cpp family the pages run: blocks of 32 values along
+ *     the head dimension, one fp16 scale d and 32 4-bit codes; with m the
+ *     value of largest magnitude (first one on ties), d = m / -8,
+ *     code = min(15, trunc(x / d + 8.5)) (0 when d = 0), value = (code - 8) d;
+ *     codes j and j + 16 share byte j (low and high nibble).  Attention for
+ *     one new token: query head h reads KV head h * Hkv / Hq (grouped
+ *     query attention), s_t = (q . k_t) / sqrt(D) over the L cached tokens,
+ *     out = sum_t softmax(s)_t v_t, in fp64 from the dequantised cache.  No
+ *     rotary embedding or mask (the pages give none; this is the product the
+ *     kernel computes).
  *  R10 ternarisation (pwwt.cn/news/5175886, section 1.2: per block, two
  *     thresholds -- values between them become 0, the two sides +1 / -1 --
  *     and a scale chosen to make the residual small; m.nxbn.cn/news/172464,
@@ -574,5 +587,85 @@ int oracle_ternarize(const float *w, int64_t N, int64_t K, int64_t ldw, int64_t 
             scales[n * G + g] = oracle_float_to_half(alpha);
         }
     }
+    return ORACLE_OK;
+}
+
+/* ------------------------------------------------------------------ */
+/* Q4_0 blocks (R12).  x: n floats (n a multiple of 32); d: n/32 fp16
+ * scale bits; qs: 16 bytes per block.                                   */
+int oracle_q4_0_quantize(const float *x, int64_t n, uint16_t *d, uint8_t *qs) {
+    if (n % 32 != 0) return ORACLE_EINVAL;
+    for (int64_t b = 0; b < n / 32; ++b) {
+        const float *v = x + 32 * b;
+        float amax = 0.0f, m = 0.0f;
+        for (int j = 0; j < 32; ++j)
+            if (fabsf(v[j]) > amax) {
+                amax = fabsf(v[j]);
+                m = v[j];
+            }
+        volatile float dd = m / -8.0f;
+        volatile float id = dd != 0.0f ? 1.0f / dd : 0.0f;
+        d[b] = oracle_float_to_half(dd);
+        for (int j = 0; j < 16; ++j) {
+            int c[2];
+            for (int h = 0; h < 2; ++h) {
+                volatile float t = v[j + 16 * h] * id;
+                volatile float u = t + 8.5f;
+                int code = (int)u; /* truncation toward zero; u >= 0.5 */
+                c[h] = code > 15 ? 15 : code;
+            }
+            qs[16 * b + j] = (uint8_t)(c[0] | (c[1] << 4));
+        }
+    }
+    return ORACLE_OK;
+}
+
+void oracle_q4_0_dequantize(const uint16_t *d, const uint8_t *qs, int64_t n, double *out) {
+    for (int64_t b = 0; b < n / 32; ++b) {
+        double s = oracle_half_to_double(d[b]);
+        for (int j = 0; j < 16; ++j) {
+            out[32 * b + j] = ((qs[16 * b + j] & 15) - 8) * s;
+            out[32 * b + j + 16] = ((qs[16 * b + j] >> 4) - 8) * s;
+        }
+    }
+}
+
+/* Decode attention (R12).  q: fp32 [Hq][D]; the cache of KV head g holds L
+ * tokens, token t's K at kd/kq block (g * L + t) * (D/32) .. (and V alike);
+ * out: fp64 [Hq][D].                                                    */
+int oracle_attention_decode(const float *q, const uint16_t *kd, const uint8_t *kq,
+                            const uint16_t *vd, const uint8_t *vq, int64_t L, int64_t Hkv,
+                            int64_t Hq, int64_t D, double *out) {
+    if (D % 32 != 0 || Hkv < 1 || Hq % Hkv != 0 || L < 1) return ORACLE_EINVAL;
+    int64_t nb = D / 32;
+    double *k = (double *)malloc((size_t)D * sizeof(double));
+    double *v = (double *)malloc((size_t)D * sizeof(double));
+    double *s = (double *)malloc((size_t)L * sizeof(double));
+    if (!k || !v || !s) { free(k); free(v); free(s); return ORACLE_EINVAL; }
+    for (int64_t h = 0; h < Hq; ++h) {
+        int64_t g = h * Hkv / Hq;
+        double smax = -INFINITY;
+        for (int64_t t = 0; t < L; ++t) {
+            int64_t blk = (g * L + t) * nb;
+            oracle_q4_0_dequantize(kd + blk, kq + 16 * blk, D, k);
+            double dot = 0.0;
+            for (int64_t i = 0; i < D; ++i) dot += (double)q[h * D + i] * k[i];
+            s[t] = dot / sqrt((double)D);
+            if (s[t] > smax) smax = s[t];
+        }
+        double z = 0.0;
+        for (int64_t i = 0; i < D; ++i) out[h * D + i] = 0.0;
+        for (int64_t t = 0; t < L; ++t) {
+            double p = exp(s[t] - smax);
+            z += p;
+            int64_t blk = (g * L + t) * nb;
+            oracle_q4_0_dequantize(vd + blk, vq + 16 * blk, D, v);
+            for (int64_t i = 0; i < D; ++i) out[h * D + i] += p * v[i];
+        }
+        for (int64_t i = 0; i < D; ++i) out[h * D + i] /= z;
+    }
+    free(k);
+    free(v);
+    free(s);
     return ORACLE_OK;
 }
