@@ -47,10 +47,14 @@ typedef enum {
     TERN_ETIMEOUT = 4      /* a bounded device-side wait ran out */
 } tern_status;
 
-/* Weight formats.  Both hold one trit per weight, t = w + 1 in {0, 1, 2}. */
+/* Weight formats.  Each holds one trit per weight, t = w + 1 in {0, 1, 2}. */
 typedef enum {
-    TERN_FMT_BASE3 = 0, /* 5 trits per byte (PTQ1_0-style), 1.6 bit/trit */
-    TERN_FMT_2BIT = 1   /* 4 trits per byte (PQ2-style), 2 bit/trit */
+    TERN_FMT_BASE3 = 0,   /* 5 trits per byte (PTQ1_0-style), 1.6 bit/trit */
+    TERN_FMT_2BIT = 1,    /* 4 trits per byte (PQ2-style), 2 bit/trit */
+    TERN_FMT_BITPLANE = 2 /* a nonzero bit and a sign bit per weight, 2 bit/trit (Bonsai
+                             page, "后面还有没有优化空间"); the format calls and the
+                             streamed entry points take it, the other compute calls
+                             return TERN_EUNSUPPORTED */
 } tern_format;
 
 /* Bit 0 of tern_matrix.flags: the packed codes and scales are not written by
@@ -77,7 +81,11 @@ typedef enum {
  *   TERN_FMT_2BIT (D2): 4-byte word w covers K in [16w, 16w+16); bits
  *     [2i, 2i+1] of byte j hold t for K = 16w + 4i + j.  Row bytes used:
  *     4*ceil(K/16).
- *   Positions past K hold t = 1 (w = 0); bytes past the used row bytes are 0.
+ *   TERN_FMT_BITPLANE (DB): 4-byte words in pairs; pair p covers K in
+ *     [32p, 32p+32): word 2p holds the nonzero bits (w != 0), word 2p+1 the
+ *     sign bits (w < 0), bit 8j + i of each for K = 32p + 4i + j.  Row bytes
+ *     used: 8*ceil(K/32).
+ *   Positions past K hold w = 0; bytes past the used row bytes are 0.
  * scales: fp16 bit patterns [N][ceil(K/group)], one per group of `group`
  * consecutive K positions of a row (the last group may be partial).
  */
@@ -139,7 +147,9 @@ tern_status tern_packed_size(int32_t fmt, int32_t N, int32_t K, int32_t group,
 
 /* Bytes per row of the canonical (file) encodings: base-3 = ceil(K/5)
  * (byte value sum_{i<5} t_i 3^i over K = 5j+i, least significant digit
- * first), 2-bit = ceil(K/4) (bits [2i,2i+1] of byte j hold K = 4j+i).  These
+ * first), 2-bit = ceil(K/4) (bits [2i,2i+1] of byte j hold K = 4j+i),
+ * bit-plane = 2*ceil(K/8) (the nonzero plane, then the sign plane, bit k mod
+ * 8 of byte k/8; the Bonsai page, "后面还有没有优化空间").  These
  * are the PTQ1_0-style (5 trits a byte) and PQ2-style (4 trits a byte) rows
  * of the Bonsai page ("Decode 为什么只能算一般", "PQ2 会不会快很多"); the
  * digit order is this library's reading, the pages give none.  Errors:
@@ -184,6 +194,29 @@ tern_status tern_import(int32_t fmt, const uint8_t *canonical, int32_t N,
  * the inverse of tern_import (same passage).  Errors as tern_unpack. */
 tern_status tern_export(const tern_matrix *W, uint8_t *canonical_out,
                         int32_t *d_invalid, void *stream);
+
+/*
+ * Producer-side ternarisation of float weights, no calibration data (page
+ * pwwt.cn/news/5175886, section 1.2: per block two thresholds -- values
+ * between them become 0, the two sides +1 and -1 -- and a scale that keeps
+ * the residual small; m.nxbn.cn/news/172464, section 1.2: threshold plus one
+ * scale per group; 4sapi page, section 三: one FP16 scale per group).  Per
+ * group of `group` (= 128) consecutive K positions of row n of w:
+ *   keep the k largest |w| (larger first, lower index first among equals),
+ *   t = sign(w) on them and 0 elsewhere, alpha = fp16(S / k) (round to
+ *   nearest even), for the k that maximises S^2 / k, S = the fp32 sum of
+ *   the kept |w| added in index order, score = fp32(fp32(S * S) / k); the
+ *   largest score wins, the smallest k among equal scores; k = 0 (t = 0,
+ *   alpha = 0) when no score is above 0.  This is the cut that minimises
+ *   sum (w - alpha t)^2 over all thresholds.
+ *  w: device fp32 [N][ldw], ldw >= K, finite values.
+ *  trits: device int8 [N][K] in {-1, 0, +1} (the input of tern_pack).
+ *  scales: device fp16 bits [N][ceil(K/128)], 2-byte aligned.
+ * Errors: TERN_EINVAL for bad shapes or pointers, TERN_EUNSUPPORTED for a
+ * group other than 128, TERN_ECUDA when the launch fails.
+ */
+tern_status tern_ternarize(const float *w, int32_t N, int32_t K, int32_t ldw, int32_t group,
+                           int8_t *trits, uint16_t *scales, void *stream);
 
 /*
  * Per-token int8 activation quantisation with an optional 128-point
@@ -371,6 +404,61 @@ tern_status tern_gateup_swiglu_streamed(const tern_matrix *Wg, const tern_matrix
 tern_status tern_gemv_streamed_noalloc(const tern_matrix *W, const float *x, int32_t ldx,
                                        int32_t qflags, int32_t M, const float *residual,
                                        float *y, int32_t ldy, void *stream);
+
+/*
+ * Q4_0 KV cache of one layer for decode attention (Bonsai page, "先交代机器和
+ * 配置": K and V cached as Q4_0; the passage before "PQ2 会不会快很多": the Q4
+ * data is decoded inside attention).  Q4_0 blocks of 32 values along the head
+ * dimension: an fp16 scale d and 32 4-bit codes, value = (code - 8) d;
+ * byte j of a block holds element j (low nibble) and element j + 16 (high
+ * nibble).  Per KV head g and token t:
+ *   k_codes[(g * capacity + t) * D/2 ..]   the D/2 code bytes of K,
+ *   k_scales[(g * capacity + t) * D/32 ..] its D/32 fp16 block scales,
+ * and v_codes / v_scales alike.  All device memory owned by the caller;
+ * codes 16-byte aligned, scales 2-byte aligned.  This build takes D = 128.
+ */
+typedef struct tern_kv_cache {
+    int32_t Hkv;       /* KV heads */
+    int32_t D;         /* head dimension (128) */
+    int32_t capacity;  /* tokens the arrays hold */
+    int32_t reserved;  /* must be 0 */
+    uint8_t *k_codes;
+    uint16_t *k_scales;
+    uint8_t *v_codes;
+    uint16_t *v_scales;
+} tern_kv_cache;
+
+/*
+ * Appends one token at position pos (< capacity): k and v are device fp32
+ * [Hkv][D] (the K and V parts of the QKV projection's output), quantised to
+ * Q4_0 with d = m / -8 (m: the value of largest magnitude in the block, the
+ * first on ties) and code = min(15, trunc(x / d + 8.5)) in fp32 (code 8 when
+ * d = 0), d stored as fp16 rounded to nearest.  Errors: TERN_EINVAL for a bad
+ * cache or position, TERN_ECUDA when a launch fails.
+ */
+tern_status tern_kv_append_q4_0(const float *k, const float *v, int32_t pos,
+                                const tern_kv_cache *cache, void *stream);
+
+/* Workspace bytes of tern_attention_decode_q4_0 for Hq query heads over L
+ * cached tokens on the current device. */
+tern_status tern_attention_workspace_bytes(int32_t Hq, int32_t L, const tern_kv_cache *cache,
+                                           size_t *bytes);
+
+/*
+ * Decode attention of one new token over the first L tokens of the cache:
+ * query head h (q: device fp32 [Hq][D]) reads KV head h * Hkv / Hq and
+ *   out[h] = sum_t softmax_t(q_h . k_t / sqrt(D)) v_t,
+ * with k_t, v_t the dequantised Q4_0 rows (no rotary embedding or mask).
+ * Split-context flash decoding: chunks of the context per CTA, merged in
+ * chunk order by a second kernel.  Hq / Hkv must be 1, 2, 4, 5 or 8.
+ *  out: device fp32 [Hq][D]; workspace: device, 16-byte aligned, at least
+ *  tern_attention_workspace_bytes() bytes (no initial contents needed).
+ * Errors: TERN_EINVAL for bad shapes, pointers or workspace,
+ * TERN_EUNSUPPORTED for D != 128 or another group size, TERN_ECUDA.
+ */
+tern_status tern_attention_decode_q4_0(const float *q, int32_t Hq, const tern_kv_cache *cache,
+                                       int32_t L, float *out, void *workspace, size_t ws_bytes,
+                                       void *stream);
 
 /*
  * Test hook of the streamed kernels (the integer dot product and the

@@ -22,7 +22,7 @@ LIBS = {
     "libtern.so": ["csrc/tern_api.cu", "csrc/tern_format.cu", "csrc/tern_quant.cu",
                    "csrc/tern_gemv.cu", "csrc/tern_gemv_tc.cu", "csrc/tern_gemv_stream.cu",
                    "csrc/tern_noalloc.cu", "csrc/tern_gemm.cu", "csrc/tern_tcdebug.cu",
-                   "csrc/tern_debug.cu"],
+                   "csrc/tern_debug.cu", "csrc/tern_ternarize.cu", "csrc/tern_attention.cu"],
     "libtern_synth.so": ["synth_csrc/tern_synth.cu"],
 }
 HEADERS = ["csrc/tern_common.cuh", "csrc/tern_internal.h", "csrc/tern_tc.cuh",

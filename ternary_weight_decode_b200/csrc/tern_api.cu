@@ -24,7 +24,9 @@ tern_status cuda_status(cudaError_t e, const char *what) {
 
 bool aligned(const void *p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
-bool valid_fmt(int32_t fmt) { return fmt == TERN_FMT_BASE3 || fmt == TERN_FMT_2BIT; }
+bool valid_fmt(int32_t fmt) {
+    return fmt == TERN_FMT_BASE3 || fmt == TERN_FMT_2BIT || fmt == TERN_FMT_BITPLANE;
+}
 
 tern_status check_matrix(const tern_matrix *W, const char *name) {
     if (!W) return fail(TERN_EINVAL, "%s: null matrix", name);
@@ -159,6 +161,76 @@ tern_status tern_export(const tern_matrix *W, uint8_t *canonical_out, int32_t *d
                        "tern_export");
 }
 
+tern_status tern_ternarize(const float *w, int32_t N, int32_t K, int32_t ldw, int32_t group,
+                           int8_t *trits, uint16_t *scales, void *stream) {
+    if (N < 1 || K < 1) return fail(TERN_EINVAL, "tern_ternarize: N and K must be >= 1%s");
+    if (group != 128) return fail(TERN_EUNSUPPORTED, "tern_ternarize: only group = 128 is supported%s");
+    if (!w || !aligned(w, 4) || ldw < K) return fail(TERN_EINVAL, "tern_ternarize: bad w or ldw%s");
+    if (!trits || !scales || !aligned(scales, 2))
+        return fail(TERN_EINVAL, "tern_ternarize: null or misaligned output%s");
+    return cuda_status(tern::launch_ternarize(w, N, K, ldw, trits, scales, static_cast<cudaStream_t>(stream)),
+                       "tern_ternarize");
+}
+
+static tern_status check_cache(const tern_kv_cache *C, const char *name) {
+    if (!C || C->Hkv < 1 || C->capacity < 1 || C->reserved != 0)
+        return fail(TERN_EINVAL, "%s: bad cache (Hkv, capacity >= 1, reserved = 0)", name);
+    if (C->D != 128) return fail(TERN_EUNSUPPORTED, "%s: this build takes head dimension 128", name);
+    if (!C->k_codes || !C->v_codes || !aligned(C->k_codes, 16) || !aligned(C->v_codes, 16) ||
+        !C->k_scales || !C->v_scales || !aligned(C->k_scales, 2) || !aligned(C->v_scales, 2))
+        return fail(TERN_EINVAL, "%s: cache arrays missing or misaligned", name);
+    return TERN_OK;
+}
+
+static cudaError_t device_sms(int *sms) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e == cudaSuccess) e = cudaDeviceGetAttribute(sms, cudaDevAttrMultiProcessorCount, dev);
+    return e;
+}
+
+tern_status tern_kv_append_q4_0(const float *k, const float *v, int32_t pos, const tern_kv_cache *cache,
+                                void *stream) {
+    tern_status st = check_cache(cache, "tern_kv_append_q4_0");
+    if (st != TERN_OK) return st;
+    if (pos < 0 || pos >= cache->capacity) return fail(TERN_EINVAL, "tern_kv_append_q4_0: pos outside the cache%s");
+    if (!k || !v || !aligned(k, 4) || !aligned(v, 4)) return fail(TERN_EINVAL, "tern_kv_append_q4_0: bad k or v%s");
+    return cuda_status(tern::launch_kv_append(k, v, pos, *cache, static_cast<cudaStream_t>(stream)),
+                       "tern_kv_append_q4_0");
+}
+
+tern_status tern_attention_workspace_bytes(int32_t Hq, int32_t L, const tern_kv_cache *cache, size_t *bytes) {
+    tern_status st = check_cache(cache, "tern_attention_workspace_bytes");
+    if (st != TERN_OK) return st;
+    if (Hq < 1 || L < 1 || !bytes) return fail(TERN_EINVAL, "tern_attention_workspace_bytes: bad arguments%s");
+    int sms = 0;
+    cudaError_t e = device_sms(&sms);
+    if (e != cudaSuccess) return cuda_status(e, "tern_attention_workspace_bytes");
+    *bytes = tern::attention_workspace_bytes(Hq, L, cache->Hkv, sms);
+    return TERN_OK;
+}
+
+tern_status tern_attention_decode_q4_0(const float *q, int32_t Hq, const tern_kv_cache *cache, int32_t L,
+                                       float *out, void *workspace, size_t ws_bytes, void *stream) {
+    const char *name = "tern_attention_decode_q4_0";
+    tern_status st = check_cache(cache, name);
+    if (st != TERN_OK) return st;
+    if (Hq < 1 || Hq % cache->Hkv != 0) return fail(TERN_EINVAL, "%s: Hq must be a multiple of Hkv", name);
+    if (L < 1 || L > cache->capacity) return fail(TERN_EINVAL, "%s: L must be in 1..capacity", name);
+    if (!q || !aligned(q, 16) || !out || !aligned(out, 4))
+        return fail(TERN_EINVAL, "%s: q (16-byte aligned) and out are required", name);
+    int sms = 0;
+    cudaError_t e = device_sms(&sms);
+    if (e != cudaSuccess) return cuda_status(e, name);
+    if (!workspace || !aligned(workspace, 16) || ws_bytes < tern::attention_workspace_bytes(Hq, L, cache->Hkv, sms))
+        return fail(TERN_EINVAL, "%s: workspace missing, misaligned or too small", name);
+    const char *why = nullptr;
+    e = tern::launch_attention(q, Hq, *cache, L, out, static_cast<float *>(workspace), sms,
+                               static_cast<cudaStream_t>(stream), &why);
+    if (why) return fail(TERN_EUNSUPPORTED, "tern_attention_decode_q4_0: %s", why);
+    return cuda_status(e, name);
+}
+
 tern_status act_quant_fwht(const void *x, int32_t x_is_fp16, int32_t M, int32_t K, int32_t ldx,
                            int32_t fwht_block, int32_t flags, int8_t *q, int32_t ldq, float *s_x,
                            void *stream) {
@@ -181,6 +253,8 @@ tern_status act_quant_fwht(const void *x, int32_t x_is_fp16, int32_t M, int32_t 
 }
 
 static tern_status run_gemv(tern::GemvLaunch &L, const char *name, cudaStream_t s) {
+    if (L.fmt == TERN_FMT_BITPLANE)
+        return fail(TERN_EUNSUPPORTED, "%s: the bit-plane format runs on the streamed entry points only", name);
     const char *why = nullptr;
     cudaError_t e = tern::launch_gemv(L, s, &why);
     if (why) return fail(TERN_EUNSUPPORTED, "%s", why);
@@ -444,6 +518,8 @@ static tern_status run_gemm(const tern_matrix *W, const int8_t *q, int32_t ldq, 
                             int32_t M, float *y, int32_t ldy, int32_t *dbg_P, void *stream) {
     tern_status st = check_matrix(W, "tern_gemm");
     if (st != TERN_OK) return st;
+    if (W->fmt == TERN_FMT_BITPLANE)
+        return fail(TERN_EUNSUPPORTED, "tern_gemm: the bit-plane format runs on the streamed entry points only%s");
     if (M < 1) return fail(TERN_EINVAL, "tern_gemm: M must be >= 1%s");
     if (!q || !aligned(q, 16) || ldq < W->K || ldq % 16 != 0)
         return fail(TERN_EINVAL, "tern_gemm: q must be 16-byte aligned with ldq >= K, ldq %% 16 == 0%s");

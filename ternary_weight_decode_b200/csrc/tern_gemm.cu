@@ -30,6 +30,16 @@
 // The per-group scale is why the accumulator is drained every 128 K: the
 // tensor cores accumulate only the exact integer partial of one group.  The
 // test-hook instantiation (DBG) also writes every partial P[m][n][g].
+//
+// Multi-token verify (Bonsai page, "后面还有没有优化空间": one weight read
+// serving several candidate tokens) runs the same kernel with a narrower
+// token tile, TM = 64 or 128 tokens (MMA N = TM), so that 17..128 token rows
+// do not pay for a 256-token tile.  When the weight-row tiles are too few to
+// fill the SMs (N = 5120: 40 tiles), a thread-block cluster of C CTAs splits
+// the superblocks of K between its ranks; each rank accumulates its groups
+// in fp32 as above, leaves its partial tile in shared memory, and rank 0
+// adds the ranks' tiles in rank order (distributed shared memory) before
+// the s_x multiply -- a fixed order, so the result does not depend on timing.
 #include "tern_gemv_common.cuh"
 #include "tern_tc.cuh"
 
@@ -37,22 +47,28 @@ namespace tern {
 namespace {
 
 constexpr int kGmTileN = 128;   // weight rows per CTA (MMA M)
-constexpr int kGmTileM = 256;   // tokens per CTA (MMA N)
 constexpr int kGmTile = 128 * 128;  // bytes of one 128 x 128 B int8 tile (codes, decoded A)
-constexpr int kGmActTile = kGmTileM * 128;  // bytes of one activation tile (kGmTileM x 128 B)
 constexpr int kGmCodeStages = 2;
 constexpr int kGmActStages = 3;
 constexpr int kGmAStages = 2;
 constexpr int kGmDecodeWarps = 4;
 constexpr int kGmEpiWarps = 16;
-constexpr int kGmEpiCols = kGmTileM * 4 / kGmEpiWarps;  // token columns per epilogue warp
 constexpr int kGmWarps = 2 + kGmDecodeWarps + kGmEpiWarps;
 constexpr int kGmThreads = 32 * kGmWarps;
 constexpr int kGmAccBufs = 2;
-constexpr int kGmTmemCols = kGmTileM * kGmAccBufs;  // kGmAccBufs accumulators of kGmTileM columns
-static_assert(kGmTmemCols <= 512, "tensor memory holds 512 columns");
 constexpr int kGmBand = 8;                     // weight-row tiles per raster band
 constexpr int kGmEpiBar = 1;                   // named barrier of the epilogue warps
+constexpr int kGmMaxSplit = 8;                 // portable cluster size
+
+// Sizes that follow from the token tile TM (MMA N): 64, 128 or 256 tokens.
+template <int TM>
+struct GmShape {
+    static_assert(TM == 64 || TM == 128 || TM == 256, "token tile");
+    static constexpr int kActTile = TM * 128;          // one TM x 128 B activation tile
+    static constexpr int kEpiCols = TM * 4 / kGmEpiWarps;  // token columns per epilogue warp
+    static constexpr int kTmemCols = TM * kGmAccBufs;  // accumulators (a power of two)
+    static_assert(kTmemCols <= 512, "tensor memory holds 512 columns");
+};
 
 struct GemmParams {
     int N, K, M, G, SB;
@@ -63,16 +79,18 @@ struct GemmParams {
     int32_t *dbg_P;  // DBG kernels only: P [M][N][G]
 };
 
+template <int TM>
 struct GemmSmem {
     uint8_t code[kGmCodeStages][kGmTile];
-    uint8_t act[kGmActStages][kGmActTile];
+    uint8_t act[kGmActStages][GmShape<TM>::kActTile];
     uint8_t a[kGmAStages][kGmTile];
     uint64_t code_full[kGmCodeStages], code_empty[kGmCodeStages];
     uint64_t act_full[kGmActStages], act_empty[kGmActStages];
     uint64_t a_full[kGmAStages], a_empty[kGmAStages];
     uint64_t acc_full[kGmAccBufs], acc_empty[kGmAccBufs];
     uint32_t tmem_base;
-    // followed by the tile's group scales, fp16 [G][128] (group-major)
+    // followed, with a split of K, by this rank's fp32 partial tile [TM][128]
+    // (token-major), then by the tile's group scales, fp16 [GL][128]
 };
 
 // w = t - 1 on four packed digits t in {0, 1, 2}: no byte carries.
@@ -118,29 +136,40 @@ __device__ __forceinline__ void decode_half(const uint32_t (&words)[32], int gg,
     }
 }
 
-template <int FMT, bool DBG>
+template <int FMT, bool DBG, int TM>
 __global__ void __launch_bounds__(kGmThreads, 1)
     gemm_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_q,
                 const GemmParams p) {
+    using Sh = GmShape<TM>;
     constexpr int GPS = FMT == TERN_FMT_BASE3 ? 5 : 4;  // groups per superblock
+    constexpr int EC = Sh::kEpiCols;
     extern __shared__ uint8_t smem_raw[];
-    GemmSmem &S = *reinterpret_cast<GemmSmem *>(
+    GemmSmem<TM> &S = *reinterpret_cast<GemmSmem<TM> *>(
         smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023));
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    // A cluster of C CTAs shares one output tile and splits its superblocks.
+    const int C = static_cast<int>(cluster_nctarank());
+    const int rank = static_cast<int>(cluster_ctarank());
+    const int tile = blockIdx.x / C;
     // Tile order: bands of kGmBand weight-row tiles, token tiles fastest
     // inside a band, so the CTAs resident at one time cover a patch of about
     // kGmBand x (148 / kGmBand) tiles: each activation tile is read by about
     // kGmBand CTAs at once, not by every weight-row tile of the grid.
-    const int tiles_n = (p.N + kGmTileN - 1) / kGmTileN, tiles_m = (p.M + kGmTileM - 1) / kGmTileM;
-    const int band = blockIdx.x / (kGmBand * tiles_m);
+    const int tiles_n = (p.N + kGmTileN - 1) / kGmTileN, tiles_m = (p.M + TM - 1) / TM;
+    const int band = tile / (kGmBand * tiles_m);
     const int band_w = min(kGmBand, tiles_n - band * kGmBand);
-    const int in_band = blockIdx.x - band * kGmBand * tiles_m;
+    const int in_band = tile - band * kGmBand * tiles_m;
     const int n0 = (band * kGmBand + in_band % band_w) * kGmTileN;
-    const int m0 = (in_band / band_w) * kGmTileM;
+    const int m0 = (in_band / band_w) * TM;
     const int G = p.G;
+    // this rank's superblocks and groups (C <= SB: every rank has some)
+    const int sb_lo = p.SB * rank / C, sb_hi = p.SB * (rank + 1) / C;
+    const int g_lo = min(G, sb_lo * GPS), g_hi = min(G, sb_hi * GPS);
+    const int GL = g_hi - g_lo;
     // After a failed wait anywhere (recorded in the device error word) the
-    // remaining CTAs leave at once instead of timing out one by one.
-    if (*reinterpret_cast<volatile int *>(&g_device_error) != 0) return;
+    // remaining CTAs leave at once instead of timing out one by one (not in
+    // a cluster, whose peers would wait for the leaver).
+    if (C == 1 && *reinterpret_cast<volatile int *>(&g_device_error) != 0) return;
 
     if (tid == 0) {
         prefetch_tmap(&tm_w);
@@ -164,7 +193,7 @@ __global__ void __launch_bounds__(kGmThreads, 1)
         fence_mbar_init();
     }
     if (warp == 1) {
-        tmem_alloc(&S.tmem_base, kGmTmemCols);
+        tmem_alloc(&S.tmem_base, Sh::kTmemCols);
         tmem_relinquish();
     }
     tc_fence_before_sync();
@@ -172,45 +201,49 @@ __global__ void __launch_bounds__(kGmThreads, 1)
     tc_fence_after_sync();
     const uint32_t tmem = S.tmem_base;
     pdl_launch_dependents();
+    // with a split of K: this rank's fp32 partial tile, at the same offset in
+    // every rank (rank 0 reads the others' through distributed shared memory)
+    float *red = reinterpret_cast<float *>(&S + 1);
+    uint16_t *ssc = reinterpret_cast<uint16_t *>(red + (C > 1 ? TM * kGmTileN : 0));
 
     if (warp == 0) {
         // ------------------------------------------------------------- TMA
         if (lane == 0) {
             pdl_wait();
-            int g = 0;
-            for (int sb = 0; sb < p.SB && g < G; ++sb) {
-                const int cs = sb % kGmCodeStages;
-                if (sb >= kGmCodeStages &&
-                    !mbar_wait_bounded(&S.code_empty[cs], ((sb / kGmCodeStages) - 1) & 1))
+            int gl = 0;
+            for (int sb = sb_lo; sb < sb_hi && gl < GL; ++sb) {
+                const int sl = sb - sb_lo, cs = sl % kGmCodeStages;
+                if (sl >= kGmCodeStages &&
+                    !mbar_wait_bounded(&S.code_empty[cs], ((sl / kGmCodeStages) - 1) & 1))
                     break;
                 mbar_arrive_expect_tx(&S.code_full[cs], kGmTile);
                 tma_load_2d_nohint(S.code[cs], &tm_w, sb * 128, n0, &S.code_full[cs]);
-                for (int gg = 0; gg < GPS && g < G; ++gg, ++g) {
-                    const int as = g % kGmActStages;
-                    if (g >= kGmActStages &&
-                        !mbar_wait_bounded(&S.act_empty[as], ((g / kGmActStages) - 1) & 1))
+                for (int gg = 0; gg < GPS && gl < GL; ++gg, ++gl) {
+                    const int as = gl % kGmActStages;
+                    if (gl >= kGmActStages &&
+                        !mbar_wait_bounded(&S.act_empty[as], ((gl / kGmActStages) - 1) & 1))
                         break;
-                    mbar_arrive_expect_tx(&S.act_full[as], kGmActTile);
-                    tma_load_2d_nohint(S.act[as], &tm_q, g * 128, m0, &S.act_full[as]);
+                    mbar_arrive_expect_tx(&S.act_full[as], Sh::kActTile);
+                    tma_load_2d_nohint(S.act[as], &tm_q, (g_lo + gl) * 128, m0, &S.act_full[as]);
                 }
             }
         }
     } else if (warp == 1) {
         // ------------------------------------------------------------- MMA
         if (lane == 0) {
-            const uint32_t idesc = idesc_i8(kGmTileN, kGmTileM, 1, 1);
-            for (int g = 0; g < G; ++g) {
-                const int as = g % kGmAStages, qs = g % kGmActStages, buf = g % kGmAccBufs;
-                bool ok = mbar_wait_bounded(&S.a_full[as], (g / kGmAStages) & 1);
-                ok = ok && mbar_wait_bounded(&S.act_full[qs], (g / kGmActStages) & 1);
-                if (g >= kGmAccBufs)
-                    ok = ok && mbar_wait_bounded(&S.acc_empty[buf], ((g / kGmAccBufs) - 1) & 1);
+            const uint32_t idesc = idesc_i8(kGmTileN, TM, 1, 1);
+            for (int gl = 0; gl < GL; ++gl) {
+                const int as = gl % kGmAStages, qs = gl % kGmActStages, buf = gl % kGmAccBufs;
+                bool ok = mbar_wait_bounded(&S.a_full[as], (gl / kGmAStages) & 1);
+                ok = ok && mbar_wait_bounded(&S.act_full[qs], (gl / kGmActStages) & 1);
+                if (gl >= kGmAccBufs)
+                    ok = ok && mbar_wait_bounded(&S.acc_empty[buf], ((gl / kGmAccBufs) - 1) & 1);
                 if (!ok) break;
                 tc_fence_after_sync();
                 const uint32_t a0 = smem_u32(S.a[as]), b0 = smem_u32(S.act[qs]);
 #pragma unroll
                 for (int s = 0; s < 4; ++s)
-                    mma_i8_ss(tmem + buf * kGmTileM, smem_desc_sw128(a0 + 32 * s),
+                    mma_i8_ss(tmem + buf * TM, smem_desc_sw128(a0 + 32 * s),
                               smem_desc_sw128(b0 + 32 * s), idesc, s > 0);
                 tc_commit(&S.acc_full[buf]);
                 tc_commit(&S.a_empty[as]);
@@ -222,11 +255,11 @@ __global__ void __launch_bounds__(kGmThreads, 1)
         const int dt = tid - 64;
         const int r = dt & (kGmTileN - 1);  // weight row of the tile
         const int half = dt >> 7;           // which 64 K of each group (warp-uniform)
-        int g = 0;
-        for (int sb = 0; sb < p.SB && g < G; ++sb) {
-            const int cs = sb % kGmCodeStages;
+        int gl = 0;
+        for (int sb = sb_lo; sb < sb_hi && gl < GL; ++sb) {
+            const int sl = sb - sb_lo, cs = sl % kGmCodeStages;
             if (!__all_sync(0xffffffffu,
-                            mbar_wait_bounded(&S.code_full[cs], (sb / kGmCodeStages) & 1)))
+                            mbar_wait_bounded(&S.code_full[cs], (sl / kGmCodeStages) & 1)))
                 break;
             uint32_t words[32];
             const uint8_t *row = S.code[cs] + r * 128;
@@ -242,11 +275,11 @@ __global__ void __launch_bounds__(kGmThreads, 1)
             if (lane == 0) mbar_arrive(&S.code_empty[cs]);
 #pragma unroll
             for (int gg = 0; gg < GPS; ++gg) {
-                if (g >= G) break;
-                const int as = g % kGmAStages;
-                if (g >= kGmAStages &&
+                if (gl >= GL) break;
+                const int as = gl % kGmAStages;
+                if (gl >= kGmAStages &&
                     !__all_sync(0xffffffffu,
-                                mbar_wait_bounded(&S.a_empty[as], ((g / kGmAStages) - 1) & 1)))
+                                mbar_wait_bounded(&S.a_empty[as], ((gl / kGmAStages) - 1) & 1)))
                     break;
                 uint8_t *arow = S.a[as] + r * 128;
                 if constexpr (kGmDecodeWarps == 4) {
@@ -260,40 +293,40 @@ __global__ void __launch_bounds__(kGmThreads, 1)
                 fence_proxy_async_smem();  // read by the tensor cores
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&S.a_full[as]);
-                ++g;
+                ++gl;
             }
         }
     } else {
         // -------------------------------------------------------- epilogue
         const int e = warp - 2 - kGmDecodeWarps;      // 0 .. kGmEpiWarps-1
         const int quarter = warp & 3;                  // tensor-memory lanes it reaches
-        const int c0 = (e >> 2) * kGmEpiCols;         // its token columns
+        const int c0 = (e >> 2) * EC;                  // its token columns
         const int r = 32 * quarter + lane;             // tile row
         const int n = n0 + r;
         const uint32_t lane_addr = static_cast<uint32_t>(32 * quarter) << 16;
-        // the tile's scales, group-major (conflict-free reads below)
-        uint16_t *ssc = reinterpret_cast<uint16_t *>(&S + 1);
-        for (int idx = tid - 32 * (2 + kGmDecodeWarps); idx < kGmTileN * G; idx += 32 * kGmEpiWarps) {
-            const int rr = idx / G, gg = idx % G;
-            ssc[gg * kGmTileN + rr] = n0 + rr < p.N ? p.scales[static_cast<int64_t>(n0 + rr) * G + gg] : 0;
+        // this rank's scales of the tile, group-major (conflict-free reads below)
+        for (int idx = tid - 32 * (2 + kGmDecodeWarps); idx < kGmTileN * GL; idx += 32 * kGmEpiWarps) {
+            const int rr = idx / GL, gg = idx % GL;
+            ssc[gg * kGmTileN + rr] =
+                n0 + rr < p.N ? p.scales[static_cast<int64_t>(n0 + rr) * G + g_lo + gg] : 0;
         }
         warpgroup_sync_n(kGmEpiBar, 32 * kGmEpiWarps);
-        float acc[kGmEpiCols];
+        float acc[EC];
 #pragma unroll
-        for (int c = 0; c < kGmEpiCols; ++c) acc[c] = 0.0f;
-        for (int g = 0; g < G; ++g) {
-            const int buf = g % kGmAccBufs;
-            const float s = __half2float(__ushort_as_half(ssc[g * kGmTileN + r]));
+        for (int c = 0; c < EC; ++c) acc[c] = 0.0f;
+        for (int gl = 0; gl < GL; ++gl) {
+            const int buf = gl % kGmAccBufs;
+            const float s = __half2float(__ushort_as_half(ssc[gl * kGmTileN + r]));
             const bool ok =
-                __all_sync(0xffffffffu, mbar_wait_bounded(&S.acc_full[buf], (g / kGmAccBufs) & 1));
+                __all_sync(0xffffffffu, mbar_wait_bounded(&S.acc_full[buf], (gl / kGmAccBufs) & 1));
             if (!ok) break;
             tc_fence_after_sync();
             uint32_t v[8];
 #pragma unroll
-            for (int h = 0; h < kGmEpiCols / 8; ++h) {
-                tmem_ld8(tmem + lane_addr + buf * kGmTileM + c0 + 8 * h, v);
+            for (int h = 0; h < EC / 8; ++h) {
+                tmem_ld8(tmem + lane_addr + buf * TM + c0 + 8 * h, v);
                 tmem_wait_ld();
-                if (h == kGmEpiCols / 8 - 1) {
+                if (h == EC / 8 - 1) {
                     tc_fence_before_sync();
                     __syncwarp();
                     if (lane == 0) mbar_arrive(&S.acc_empty[buf]);
@@ -307,25 +340,49 @@ __global__ void __launch_bounds__(kGmThreads, 1)
                     for (int c = 0; c < 8; ++c) {
                         const int m = m0 + c0 + 8 * h + c;
                         if (m < p.M && n < p.N)
-                            p.dbg_P[(static_cast<int64_t>(m) * p.N + n) * G + g] = static_cast<int>(v[c]);
+                            p.dbg_P[(static_cast<int64_t>(m) * p.N + n) * G + g_lo + gl] =
+                                static_cast<int>(v[c]);
                     }
                 }
             }
         }
-        pdl_wait();  // s_x comes from the previous kernel
-        if (n < p.N) {
+        if (C == 1) {
+            pdl_wait();  // s_x comes from the previous kernel
+            if (n < p.N) {
 #pragma unroll
-            for (int c = 0; c < kGmEpiCols; ++c) {
-                const int m = m0 + c0 + c;
-                if (m < p.M) p.y[static_cast<int64_t>(m) * p.ldy + n] = __ldg(p.s_x + m) * acc[c];
+                for (int c = 0; c < EC; ++c) {
+                    const int m = m0 + c0 + c;
+                    if (m < p.M) p.y[static_cast<int64_t>(m) * p.ldy + n] = __ldg(p.s_x + m) * acc[c];
+                }
             }
+        } else {
+            // this rank's partial tile, token-major (lanes write consecutive rows)
+#pragma unroll
+            for (int c = 0; c < EC; ++c) red[(c0 + c) * kGmTileN + r] = acc[c];
         }
     }
     tc_fence_before_sync();
     __syncthreads();
+    if (C > 1) {
+        cluster_sync();  // every rank's partial tile is in its shared memory
+        if (rank == 0 && warp >= 2 + kGmDecodeWarps) {
+            const int e = warp - 2 - kGmDecodeWarps;
+            const int c0 = (e >> 2) * EC, r = 32 * (warp & 3) + lane, n = n0 + r;
+            pdl_wait();
+#pragma unroll 4
+            for (int c = 0; c < EC; ++c) {
+                float* own = red + (c0 + c) * kGmTileN + r;
+                float v = *own;
+                for (int q = 1; q < C; ++q) v += ld_shared_cluster_f32(map_shared_rank(own, q));
+                const int m = m0 + c0 + c;
+                if (n < p.N && m < p.M) p.y[static_cast<int64_t>(m) * p.ldy + n] = __ldg(p.s_x + m) * v;
+            }
+        }
+        cluster_sync();  // peers keep their shared memory until rank 0 has read it
+    }
     if (warp == 1) {
         tc_fence_after_sync();
-        tmem_dealloc(tmem, kGmTmemCols);
+        tmem_dealloc(tmem, Sh::kTmemCols);
     }
 }
 
@@ -334,9 +391,75 @@ bool make_tmap_2d(CUtensorMap *map, const void *base, uint64_t inner, uint64_t r
     return make_u8_tmap_2d(map, base, inner, rows, stride, 128, box_rows);
 }
 
-size_t gemm_smem_bytes(int G) { return sizeof(GemmSmem) + static_cast<size_t>(G) * kGmTileN * 2 + 1024; }
+template <int TM>
+size_t gemm_smem_bytes(int GL, bool split) {
+    return sizeof(GemmSmem<TM>) + (split ? static_cast<size_t>(TM) * kGmTileN * 4 : 0) +
+           static_cast<size_t>(GL) * kGmTileN * 2 + 1024;
+}
+
+template <int TM>
+cudaError_t launch_gemm_tm(const GemmLaunch &L, const GemmParams &p, int C, cudaStream_t s,
+                           const char **why) {
+    CUtensorMap tm_w, tm_q;
+    if (!make_tmap_2d(&tm_w, L.packed, static_cast<uint64_t>(L.row_bytes), static_cast<uint64_t>(L.N),
+                      static_cast<uint64_t>(L.row_stride), kGmTileN) ||
+        !make_tmap_2d(&tm_q, L.q, static_cast<uint64_t>(L.K), static_cast<uint64_t>(L.M),
+                      static_cast<uint64_t>(L.ldq), TM)) {
+        *why = "cuTensorMapEncodeTiled failed or is unavailable";
+        return cudaErrorInvalidValue;
+    }
+    const int GPS = L.fmt == TERN_FMT_BASE3 ? 5 : 4;
+    const int per_rank = static_cast<int>(ceil_div(p.SB, C)) * GPS;  // groups of the widest rank
+    const int GL_max = per_rank < p.G ? per_rank : p.G;
+    const size_t smem = gemm_smem_bytes<TM>(GL_max, C > 1);
+    if (smem > 227 * 1024) {
+        *why = "K too large for the shared-memory scale block of the prefill GEMM (K <= 40960)";
+        return cudaErrorInvalidValue;
+    }
+    auto kern = L.dbg_P ? (L.fmt == TERN_FMT_BASE3 ? gemm_kernel<TERN_FMT_BASE3, true, TM>
+                                                   : gemm_kernel<TERN_FMT_2BIT, true, TM>)
+                        : (L.fmt == TERN_FMT_BASE3 ? gemm_kernel<TERN_FMT_BASE3, false, TM>
+                                                   : gemm_kernel<TERN_FMT_2BIT, false, TM>);
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(smem));
+    if (e != cudaSuccess) return e;
+    const long long tiles = ceil_div(L.N, kGmTileN) * ceil_div(L.M, TM);
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(tiles * C), 1, 1);
+    cfg.blockDim = dim3(kGmThreads, 1, 1);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    attr[1].id = cudaLaunchAttributeClusterDimension;
+    attr[1].val.clusterDim.x = C;
+    attr[1].val.clusterDim.y = 1;
+    attr[1].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = C > 1 ? 2 : 1;
+    e = cudaLaunchKernelEx(&cfg, kern, tm_w, tm_q, p);
+    if (e != cudaSuccess) return e;
+    return cudaGetLastError();
+}
 
 }  // namespace
+
+// Token tile and split of K for M token rows: the narrowest tile that holds
+// them (64, 128; 256 beyond), and, for TM <= 128, a cluster split of K when
+// the output tiles alone would leave most SMs idle.
+void gemm_plan(int N, int M, int SB, int num_sms, int *TM, int *C) {
+    *TM = M <= 64 ? 64 : (M <= 128 ? 128 : 256);
+    *C = 1;
+    const long long tiles = ceil_div(N, kGmTileN) * ceil_div(M, *TM);
+    if (*TM <= 128 && tiles * 3 < 2LL * num_sms) {
+        long long c = num_sms / tiles;
+        if (c > kGmMaxSplit) c = kGmMaxSplit;
+        if (c > SB) c = SB;
+        if (c < 1) c = 1;
+        *C = static_cast<int>(c);
+    }
+}
 
 cudaError_t launch_gemm(const GemmLaunch &L, cudaStream_t s, const char **why) {
     GemmParams p = {};
@@ -350,39 +473,15 @@ cudaError_t launch_gemm(const GemmLaunch &L, cudaStream_t s, const char **why) {
     p.y = L.y;
     p.ldy = L.ldy;
     p.dbg_P = L.dbg_P;
-    CUtensorMap tm_w, tm_q;
-    if (!make_tmap_2d(&tm_w, L.packed, static_cast<uint64_t>(L.row_bytes), static_cast<uint64_t>(L.N),
-                      static_cast<uint64_t>(L.row_stride), kGmTileN) ||
-        !make_tmap_2d(&tm_q, L.q, static_cast<uint64_t>(L.K), static_cast<uint64_t>(L.M),
-                      static_cast<uint64_t>(L.ldq), kGmTileM)) {
-        *why = "cuTensorMapEncodeTiled failed or is unavailable";
-        return cudaErrorInvalidValue;
-    }
-    const size_t smem = gemm_smem_bytes(p.G);
-    if (smem > 227 * 1024) {
-        *why = "K too large for the shared-memory scale block of the prefill GEMM (K <= 40960)";
-        return cudaErrorInvalidValue;
-    }
-    cudaError_t e;
-    auto kern = L.dbg_P ? (L.fmt == TERN_FMT_BASE3 ? gemm_kernel<TERN_FMT_BASE3, true>
-                                                   : gemm_kernel<TERN_FMT_2BIT, true>)
-                        : (L.fmt == TERN_FMT_BASE3 ? gemm_kernel<TERN_FMT_BASE3, false>
-                                                   : gemm_kernel<TERN_FMT_2BIT, false>);
-    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+    int dev = 0, sms = 148;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     if (e != cudaSuccess) return e;
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(static_cast<unsigned>(ceil_div(L.N, kGmTileN) * ceil_div(L.M, kGmTileM)), 1, 1);
-    cfg.blockDim = dim3(kGmThreads, 1, 1);
-    cfg.dynamicSmemBytes = smem;
-    cfg.stream = s;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    e = cudaLaunchKernelEx(&cfg, kern, tm_w, tm_q, p);
-    if (e != cudaSuccess) return e;
-    return cudaGetLastError();
+    int TM = 256, C = 1;
+    gemm_plan(L.N, L.M, p.SB, sms, &TM, &C);
+    if (TM == 64) return launch_gemm_tm<64>(L, p, C, s, why);
+    if (TM == 128) return launch_gemm_tm<128>(L, p, C, s, why);
+    return launch_gemm_tm<256>(L, p, C, s, why);
 }
 
 }  // namespace tern

@@ -34,6 +34,11 @@ struct Fmt<TERN_FMT_2BIT> {
     static constexpr int kPos = 512;
     static constexpr int kGroups = 4;
 };
+template <>
+struct Fmt<TERN_FMT_BITPLANE> {  // the streamed kernels only
+    static constexpr int kPos = 512;
+    static constexpr int kGroups = 4;
+};
 
 struct GemvParams {
     int N, K, G;

@@ -150,9 +150,10 @@ __device__ __forceinline__ void sk_item(Words4 words4, const float (&sc)[Fmt<FMT
         acc[m] = 0;
         yacc[m] = 0.0f;
     }
-    // sum w q = sum t q - sum q over the group (t = w + 1)
+    // sum w q = sum t q - sum q over the group (t = w + 1); the bit-plane
+    // path accumulates sum w q itself
     auto finish = [&](int m, int g) {
-        const int P = acc[m] - sq_sb[(m * GT + g) * 4];
+        const int P = FMT == TERN_FMT_BITPLANE ? acc[m] : acc[m] - sq_sb[(m * GT + g) * 4];
         sink(m, g, P);
         yacc[m] = fmaf(sc[g], static_cast<float>(P), yacc[m]);
         acc[m] = 0;
@@ -188,6 +189,42 @@ __device__ __forceinline__ void sk_item(Words4 words4, const float (&sc)[Fmt<FMT
                     if (dd > 0 && (dd & 31) == 0) finish(m, (dd >> 5) - 1);
                     acc[m] = dp4a_ss(t[d], aw[d], acc[m]);
                 }
+            }
+        } else if constexpr (FMT == TERN_FMT_BITPLANE) {
+            // two word pairs (nonzero n, sign s) of 32 positions: bit 8j + i
+            // of a word is position 4i + j of its pair, so the masked word
+            // n & (0x01010101 << i) is 2^i times a 0/1 byte vector aligned
+            // with activation word i; w = n (1 - 2 s).
+#pragma unroll
+            for (int m = 0; m < MT; ++m) {
+                const uint8_t *a = act_sb + m * Kpad + c * 64;
+                uint32_t aw[16];
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    const uint4 v = lds128(a + 16 * j);
+                    aw[4 * j + 0] = v.x;
+                    aw[4 * j + 1] = v.y;
+                    aw[4 * j + 2] = v.z;
+                    aw[4 * j + 3] = v.w;
+                }
+                int an[8] = {0, 0, 0, 0, 0, 0, 0, 0}, as[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+#pragma unroll
+                for (int pr = 0; pr < 2; ++pr) {
+                    const uint32_t nz = words[2 * pr], ng = words[2 * pr] & words[2 * pr + 1];
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) {
+                        an[i] = dp4a_us(nz & (0x01010101u << i), aw[8 * pr + i], an[i]);
+                        as[i] = dp4a_us(ng & (0x01010101u << i), aw[8 * pr + i], as[i]);
+                    }
+                }
+                int sn = 0, sg = 0;
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    sn += an[i] >> i;  // exact: an[i] is a multiple of 2^i
+                    sg += as[i] >> i;
+                }
+                acc[m] += sn - 2 * sg;
+                if (c & 1) finish(m, c >> 1);
             }
         } else {
 #pragma unroll
@@ -903,6 +940,9 @@ cudaError_t launch_sk_any(const StreamLaunch &S, cudaStream_t s, const char **wh
     if (S.fmt == TERN_FMT_BASE3)
         return S.swiglu ? launch_sk_mt<TERN_FMT_BASE3, kModeSwiglu, DBG>(S, s, why)
                         : launch_sk_mt<TERN_FMT_BASE3, kModeGemv, DBG>(S, s, why);
+    if (S.fmt == TERN_FMT_BITPLANE)
+        return S.swiglu ? launch_sk_mt<TERN_FMT_BITPLANE, kModeSwiglu, DBG>(S, s, why)
+                        : launch_sk_mt<TERN_FMT_BITPLANE, kModeGemv, DBG>(S, s, why);
     return S.swiglu ? launch_sk_mt<TERN_FMT_2BIT, kModeSwiglu, DBG>(S, s, why)
                     : launch_sk_mt<TERN_FMT_2BIT, kModeGemv, DBG>(S, s, why);
 }

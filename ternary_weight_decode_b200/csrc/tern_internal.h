@@ -50,12 +50,14 @@ inline cudaError_t current_device(int *dev) {
 inline int64_t device_row_bytes(int fmt, int64_t K) {
     if (fmt == TERN_FMT_BASE3) return 4 * ((K + 19) / 20);
     if (fmt == TERN_FMT_2BIT) return 4 * ((K + 15) / 16);
+    if (fmt == TERN_FMT_BITPLANE) return 8 * ((K + 31) / 32);
     return -1;
 }
 
 inline int64_t canonical_row_bytes(int fmt, int64_t K) {
     if (fmt == TERN_FMT_BASE3) return (K + 4) / 5;
     if (fmt == TERN_FMT_2BIT) return (K + 3) / 4;
+    if (fmt == TERN_FMT_BITPLANE) return 2 * ((K + 7) / 8);
     return -1;
 }
 
@@ -76,6 +78,18 @@ inline int64_t tiled_scales_bytes(int fmt, int64_t N, int64_t K) {
     const int64_t gps = (fmt == TERN_FMT_BASE3) ? 5 : 4;
     return ceil_div(N, 32) * SB * 32 * gps * 2;
 }
+
+// ---------------------------------------------------------------- ternarisation
+cudaError_t launch_ternarize(const float *w, int N, int K, int ldw, int8_t *trits, uint16_t *scales,
+                             cudaStream_t s);
+
+// ---------------------------------------------------------------- attention
+cudaError_t launch_kv_append(const float *k, const float *v, int pos, const tern_kv_cache &C,
+                             cudaStream_t s);
+int attention_chunk(int L, int Hkv, int num_sms);
+size_t attention_workspace_bytes(int Hq, int L, int Hkv, int num_sms);
+cudaError_t launch_attention(const float *q, int Hq, const tern_kv_cache &C, int L, float *out,
+                             float *part, int num_sms, cudaStream_t s, const char **why);
 
 // ---------------------------------------------------------------- quant
 cudaError_t launch_act_quant(const void *x, bool fp16, int M, int K, int ldx, int fwht_block,
@@ -178,6 +192,9 @@ struct GemmLaunch {
     int32_t *dbg_P;  // test hook only: exact int32 group partials [M][N][ceil(K/128)]
 };
 cudaError_t launch_gemm(const GemmLaunch &L, cudaStream_t s, const char **why);
+// Token tile (64, 128 or 256 tokens) and cluster split of K of tern_gemm for
+// an N x K matrix (SB superblocks) and M token rows.
+void gemm_plan(int N, int M, int SB, int num_sms, int *TM, int *C);
 
 // Sets the message tern_last_error() returns on the calling host thread.
 tern_status set_last_error(tern_status s, const char *message);

@@ -141,6 +141,19 @@ def activation_rows(seeds, K: int) -> np.ndarray:
     return np.concatenate([activations(int(s), 1, K) for s in seeds], axis=0)
 
 
+def float_weights(seed: int, N: int, K: int) -> np.ndarray:
+    """fp32 weights [N, K] for the ternariser: N(0, 0.02) with 1% of the
+    entries x10, every 7th row rounded to a coarse grid (repeated magnitudes,
+    so that ties occur), and row 3 (when present) all zero."""
+    rng = np.random.default_rng(seed)
+    w = rng.standard_normal((N, K)) * 0.02
+    w[rng.random((N, K)) < 0.01] *= 10.0
+    w[::7] = np.round(w[::7] * 200.0) / 200.0
+    if N > 3:
+        w[3] = 0.0
+    return w.astype(np.float32)
+
+
 def groups(K: int, group: int = 128) -> int:
     return (K + group - 1) // group
 

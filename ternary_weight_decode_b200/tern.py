@@ -19,7 +19,7 @@ _PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_PKG, "libtern.so")
 
 TERN_OK, TERN_EINVAL, TERN_ECUDA, TERN_EUNSUPPORTED, TERN_ETIMEOUT = 0, 1, 2, 3, 4
-TERN_FMT_BASE3, TERN_FMT_2BIT = 0, 1
+TERN_FMT_BASE3, TERN_FMT_2BIT, TERN_FMT_BITPLANE = 0, 1, 2
 TERN_MATRIX_STATIC = 1
 TERN_QUANT_RMSNORM = 1
 TERN_QUANT_FWHT128 = 2
@@ -44,6 +44,19 @@ class tern_matrix(ctypes.Structure):
         ("scales_tiled", ctypes.c_void_p),
         ("flags", ctypes.c_int32),
         ("reserved", ctypes.c_int32),
+    ]
+
+
+class tern_kv_cache(ctypes.Structure):
+    _fields_ = [
+        ("Hkv", ctypes.c_int32),
+        ("D", ctypes.c_int32),
+        ("capacity", ctypes.c_int32),
+        ("reserved", ctypes.c_int32),
+        ("k_codes", ctypes.c_void_p),
+        ("k_scales", ctypes.c_void_p),
+        ("v_codes", ctypes.c_void_p),
+        ("v_scales", ctypes.c_void_p),
     ]
 
 
@@ -76,6 +89,7 @@ def lib() -> ctypes.CDLL:
                 "tern_import": (ctypes.c_int, [i32, p, i32, i32, p, i64, p, p]),
                 "tern_export": (ctypes.c_int, [pm, p, p, p]),
                 "act_quant_fwht": (ctypes.c_int, [p, i32, i32, i32, i32, i32, i32, p, i32, p, p]),
+                "tern_ternarize": (ctypes.c_int, [p, i32, i32, i32, i32, p, p, p]),
                 "tern_gemv": (ctypes.c_int, [pm, p, i32, p, i32, p, p, i32, p]),
                 "tern_gateup_swiglu": (ctypes.c_int, [pm, pm, p, i32, p, i32, p, i32, p]),
                 "tern_debug_group_partials": (ctypes.c_int, [pm, p, i32, i32, p, p]),
@@ -93,6 +107,11 @@ def lib() -> ctypes.CDLL:
                                                        p, sz, p]),
                 "tern_debug_gemm_partials": (ctypes.c_int, [pm, p, i32, p, i32, p, i32, p, p]),
                 "tern_debug_bounded_wait": (ctypes.c_int, [i32, i64, p]),
+                "tern_kv_append_q4_0": (ctypes.c_int, [p, p, i32, ctypes.POINTER(tern_kv_cache), p]),
+                "tern_attention_workspace_bytes": (ctypes.c_int, [i32, i32, ctypes.POINTER(tern_kv_cache),
+                                                                  ctypes.POINTER(sz)]),
+                "tern_attention_decode_q4_0": (ctypes.c_int, [p, i32, ctypes.POINTER(tern_kv_cache), i32, p,
+                                                              p, sz, p]),
                 "tern_gemv_fused": (ctypes.c_int, [pm, p, i32, p, i32, i32, i32, p, p, i32, p, i32, p]),
                 "tern_gateup_swiglu_fused": (ctypes.c_int, [pm, pm, p, i32, p, i32, i32, i32, p, i32,
                                                             p, i32, p]),
@@ -216,6 +235,18 @@ def tern_export(W: TernMatrix, canonical_out: torch.Tensor, d_invalid=None, stre
     s = W.struct()
     _check(lib().tern_export(ctypes.byref(s), _ptr(canonical_out), _ptr(d_invalid),
                              _stream(stream)), "tern_export")
+
+
+def tern_ternarize(w: torch.Tensor, trits: torch.Tensor, scales: torch.Tensor, K: int | None = None,
+                   stream=None):
+    """fp32 weights w [N, >=K] -> trits int8 [N, K] and fp16 group scales [N, G]."""
+    assert w.dtype == torch.float32 and w.stride(1) == 1
+    N = w.shape[0]
+    K = w.shape[1] if K is None else K
+    assert trits.dtype == torch.int8 and trits.is_contiguous() and trits.shape == (N, K)
+    assert scales.dtype == torch.float16 and scales.is_contiguous()
+    _check(lib().tern_ternarize(_ptr(w), N, K, w.stride(0), GROUP, _ptr(trits), _ptr(scales),
+                                _stream(stream)), "tern_ternarize")
 
 
 # ------------------------------------------------------------------ compute
@@ -418,6 +449,64 @@ def tern_debug_bounded_wait(kind: int, budget_cycles: int, stream=None):
     """Test hook: a kernel whose bounded wait (0: mbarrier, 1: tagged word) runs out."""
     _check(lib().tern_debug_bounded_wait(kind, budget_cycles, _stream(stream)),
            "tern_debug_bounded_wait")
+
+
+@dataclass
+class KVCache:
+    """A Q4_0 KV cache of one layer: codes uint8 [Hkv, capacity, D/2] and
+    fp16 scales [Hkv, capacity, D/32] for K and for V."""
+    Hkv: int
+    D: int
+    capacity: int
+    k_codes: torch.Tensor
+    k_scales: torch.Tensor
+    v_codes: torch.Tensor
+    v_scales: torch.Tensor
+
+    @staticmethod
+    def empty(Hkv: int, D: int, capacity: int, device="cuda") -> "KVCache":
+        def codes():
+            return torch.zeros((Hkv, capacity, D // 2), dtype=torch.uint8, device=device)
+
+        def scales():
+            return torch.zeros((Hkv, capacity, D // 32), dtype=torch.float16, device=device)
+        return KVCache(Hkv, D, capacity, codes(), scales(), codes(), scales())
+
+    def struct(self) -> tern_kv_cache:
+        return tern_kv_cache(self.Hkv, self.D, self.capacity, 0, self.k_codes.data_ptr(),
+                             self.k_scales.data_ptr(), self.v_codes.data_ptr(), self.v_scales.data_ptr())
+
+
+def tern_kv_append_q4_0(k: torch.Tensor, v: torch.Tensor, pos: int, cache: KVCache, stream=None):
+    """Quantises one token's k and v (fp32 [Hkv, D]) into the cache at pos."""
+    assert k.dtype == torch.float32 and v.dtype == torch.float32 and k.is_contiguous() and v.is_contiguous()
+    c = cache.struct()
+    _check(lib().tern_kv_append_q4_0(_ptr(k), _ptr(v), pos, ctypes.byref(c), _stream(stream)),
+           "tern_kv_append_q4_0")
+
+
+def tern_attention_workspace_bytes(Hq: int, L: int, cache: KVCache) -> int:
+    b = ctypes.c_size_t()
+    c = cache.struct()
+    _check(lib().tern_attention_workspace_bytes(Hq, L, ctypes.byref(c), ctypes.byref(b)),
+           "tern_attention_workspace_bytes")
+    return b.value
+
+
+def attention_workspace(Hq: int, L: int, cache: KVCache) -> torch.Tensor:
+    n = tern_attention_workspace_bytes(Hq, L, cache)
+    return torch.empty(((n + 15) // 16) * 4, dtype=torch.float32, device=cache.k_codes.device)
+
+
+def tern_attention_decode_q4_0(q: torch.Tensor, cache: KVCache, L: int, out: torch.Tensor,
+                               workspace: torch.Tensor, stream=None):
+    """out fp32 [Hq, D] = attention of q fp32 [Hq, D] over the first L cached tokens."""
+    assert q.dtype == torch.float32 and q.is_contiguous() and out.dtype == torch.float32
+    Hq = q.shape[0]
+    c = cache.struct()
+    _check(lib().tern_attention_decode_q4_0(_ptr(q), Hq, ctypes.byref(c), L, _ptr(out), _ptr(workspace),
+                                            workspace.numel() * workspace.element_size(),
+                                            _stream(stream)), "tern_attention_decode_q4_0")
 
 
 ENGINE_TENSOR_CORES, ENGINE_CUDA_CORES = 0, 1

@@ -98,7 +98,7 @@ def test_pack_rejects_bad_stride_and_sizes():
     lib = _lib()
     assert lib.tern_pack(0, ctypes.c_void_p(4096), 4, 256, ctypes.c_void_p(4096), 48, None, None) == 1
     assert lib.tern_pack(0, ctypes.c_void_p(4096), 0, 256, ctypes.c_void_p(4096), 64, None, None) == 1
-    assert lib.tern_pack(2, ctypes.c_void_p(4096), 4, 256, ctypes.c_void_p(4096), 64, None, None) == 1
+    assert lib.tern_pack(3, ctypes.c_void_p(4096), 4, 256, ctypes.c_void_p(4096), 64, None, None) == 1
 
 
 def test_packed_size_matches_layout():
@@ -162,3 +162,4 @@ def test_noalloc_validates_before_touching_its_array():
     st = lib.tern_gemv_streamed_noalloc(ctypes.byref(m), ctypes.c_void_p(4096), 256, 8, 1, None,
                                         ctypes.c_void_p(4096), 4, None)
     assert st == 1 and b"qflags" in lib.tern_last_error()
+

@@ -13,7 +13,15 @@ SHAPES = [(1, 1), (3, 5), (7, 19), (9, 20), (5, 21), (33, 127), (40, 300), (17, 
           (8, 17408)]
 
 
-@pytest.mark.parametrize("fmt", [tern.TERN_FMT_BASE3, tern.TERN_FMT_2BIT])
+ALL_FMTS = [tern.TERN_FMT_BASE3, tern.TERN_FMT_2BIT, tern.TERN_FMT_BITPLANE]
+
+
+def canonical(fmt, w):
+    return {tern.TERN_FMT_BASE3: oracle.pack_base3, tern.TERN_FMT_2BIT: oracle.pack_2bit,
+            tern.TERN_FMT_BITPLANE: oracle.pack_bitplane}[fmt](w)
+
+
+@pytest.mark.parametrize("fmt", ALL_FMTS)
 @pytest.mark.parametrize("N,K", SHAPES)
 def test_pack_matches_oracle_device_layout(fmt, N, K):
     w = synth.trits(11, 2, N, K)
@@ -30,11 +38,11 @@ def test_pack_matches_oracle_device_layout(fmt, N, K):
     assert int(bad.item()) == 0
 
 
-@pytest.mark.parametrize("fmt", [tern.TERN_FMT_BASE3, tern.TERN_FMT_2BIT])
+@pytest.mark.parametrize("fmt", ALL_FMTS)
 @pytest.mark.parametrize("N,K", SHAPES)
 def test_import_export_canonical(fmt, N, K):
     w = synth.trits(12, 4, N, K)
-    canon = oracle.pack_base3(w) if fmt == tern.TERN_FMT_BASE3 else oracle.pack_2bit(w)
+    canon = canonical(fmt, w)
     M = tern.TernMatrix.empty(fmt, N, K)
     bad = torch.zeros(1, dtype=torch.int32, device="cuda")
     tern.tern_import(fmt, to_dev(canon), K, M, d_invalid=bad)
@@ -83,3 +91,40 @@ def test_device_generator_matches_host():
             synth.scales(seed, stream + 1, N, 8).view(np.uint16))
     rows = synth.device_trits(3, 9, 4, K, row0=150).cpu().numpy()
     np.testing.assert_array_equal(rows, synth.trits_rows(3, 9, np.arange(150, 154), K))
+
+
+def test_bitplane_invalid_bits_are_counted():
+    """A sign bit without its nonzero bit, in the device layout and in the
+    canonical planes, and a nonzero bit past K, are counted and read as 0."""
+    K = 40
+    w = np.zeros((1, K), np.int8)
+    M = tern.TernMatrix.empty(tern.TERN_FMT_BITPLANE, 1, K)
+    tern.tern_pack(tern.TERN_FMT_BITPLANE, to_dev(w), M)
+    raw = M.packed.cpu().numpy()
+    raw[0, 4] |= 1           # sign word of pair 0: position 0 has no nonzero bit
+    raw[0, 8 + 3] |= 0x80    # nonzero word of pair 1, bit 31: position 32 + 28 + 3 = 63 >= K
+    M.packed.copy_(torch.from_numpy(raw))
+    bad = torch.zeros(1, dtype=torch.int32, device="cuda")
+    out = torch.full((1, K), 9, dtype=torch.int8, device="cuda")
+    tern.tern_unpack(M, out, d_invalid=bad)
+    assert int(bad.item()) == 2 and not out.cpu().numpy().any()
+    canon = oracle.pack_bitplane(w)
+    canon[0, 5 + 1] |= 2     # sign plane, position 9, nonzero bit clear
+    bad.zero_()
+    tern.tern_import(tern.TERN_FMT_BITPLANE, to_dev(canon), K, M, d_invalid=bad)
+    assert int(bad.item()) == 1
+
+
+def test_bitplane_rejected_by_the_non_streamed_kernels():
+    N, K = 64, 256
+    w = synth.trits(13, 0, N, K)
+    M = make_matrix(tern.TERN_FMT_BITPLANE, w, synth.scales(13, 1, N, 2))
+    q = torch.zeros((1, K), dtype=torch.int8, device="cuda")
+    s = torch.ones(1, dtype=torch.float32, device="cuda")
+    y = torch.zeros((1, N), dtype=torch.float32, device="cuda")
+    with pytest.raises(tern.TernError) as e:
+        tern.tern_gemv(M, q, s, y)
+    assert e.value.status == tern.TERN_EUNSUPPORTED
+    with pytest.raises(tern.TernError) as e:
+        tern.tern_gemm(M, q, s, y)
+    assert e.value.status == tern.TERN_EUNSUPPORTED

@@ -96,3 +96,50 @@ def test_gemm_prefill_shapes_sampled(fmt, K, N, M):
     ref = oracle.gemv(w, sw, q[toks], s[toks])
     assert np.max(np.abs(got - ref)) <= tolerance(ref)
     assert tern.tern_device_error() == 0
+
+
+# ---------------------------------------------------------------- multi-token verify
+@pytest.mark.parametrize("fmt", FMTS)
+@pytest.mark.parametrize("N,K,M", [(300, 5120, 17), (512, 17408, 100), (1000, 1280, 64),
+                                   (130, 5120, 128), (5120, 640, 65), (2000, 17408, 33)])
+def test_verify_sizes_match_oracle(fmt, N, K, M):
+    """Token rows 17..128 run on 64- or 128-token tiles, with a cluster split
+    of K when the weight-row tiles are few (N = 300, 512, 130: up to 8 ranks)."""
+    w = synth.trits(N + 3 * K, 0, N, K)
+    sw = synth.scales(N + 3 * K, 1, N, synth.groups(K))
+    q, s = quantised(N + 7 * M, M, K)
+    W = make_matrix(fmt, w, sw)
+    ldq = ((K + 15) // 16) * 16
+    y = torch.full((M + 2, N + 3), 77.0, dtype=torch.float32, device="cuda")
+    tern.tern_gemm(W, padded_q(q, ldq), to_dev(s), y, M=M)
+    ref = oracle.gemv(w, sw, q, s)
+    got = y.cpu().numpy()
+    assert np.max(np.abs(got[:M, :N] - ref)) <= tolerance(ref)
+    assert (got[:M, N:] == 77.0).all() and (got[M:] == 77.0).all()
+    # the same launch with its partials: exact integers on every rank
+    P = torch.full((M, N, synth.groups(K)), -(1 << 30), dtype=torch.int32, device="cuda")
+    y2 = torch.zeros((M, N), dtype=torch.float32, device="cuda")
+    tern.tern_debug_gemm_partials(W, padded_q(q, ldq), to_dev(s), y2, P, M=M)
+    np.testing.assert_array_equal(P.cpu().numpy(), oracle.group_partials(w, q))
+    np.testing.assert_array_equal(y2.cpu().numpy(), got[:M, :N])
+    assert tern.tern_device_error() == 0
+
+
+@pytest.mark.parametrize("fmt", FMTS)
+@pytest.mark.parametrize("K,N,M", [(5120, 17408, 64), (17408, 5120, 128), (17408, 5120, 24)])
+def test_verify_full_shapes_sampled(fmt, K, N, M):
+    """The 27B-shaped gate/up and down matrices at verify sizes, in the
+    launch configuration the bench times, checked on sampled rows."""
+    seed = 90 + M
+    W = big_matrix(fmt, N, K, seed)
+    q, s = quantised(seed, M, K)
+    y = torch.empty((M, N), dtype=torch.float32, device="cuda")
+    tern.tern_gemm(W, to_dev(q), to_dev(s), y)
+    rng = np.random.default_rng(M)
+    rows = np.unique(np.concatenate([[0, N - 1, 127, 128, 4095], rng.integers(0, N, 80)]))
+    got = y[:, torch.from_numpy(rows).cuda()].cpu().numpy()
+    w = synth.trits_rows(seed, 0, rows, K)
+    sw = synth.scales_rows(seed, 1, rows, synth.groups(K))
+    ref = oracle.gemv(w, sw, q, s)
+    assert np.max(np.abs(got - ref)) <= tolerance(ref)
+    assert tern.tern_device_error() == 0
