@@ -17,7 +17,9 @@
 //    (its codes as four 16-byte loads), sum_b d_b (sum_i q_i c_i - 8 sum_i q_i)
 //    with the per-block query sums precomputed.  Values: a warp per token, a
 //    lane per four dimensions, p_t d_b (c - 8) accumulated in fp32.  The CTA
-//    writes its chunk's max score, exp-sum and unnormalised output.
+//    writes its chunk's max score, exp-sum and unnormalised output.  Chunks
+//    are sized for about eight resident CTAs per SM, so the loads of many
+//    warps are in flight at once.
 //  * attn_combine_kernel: per query head, the chunks' partial results merged
 //    in chunk order with the running-max rule (a fixed order: the result
 //    does not depend on timing).
@@ -175,17 +177,34 @@ __global__ void __launch_bounds__(kAttThreads)
         const int word = (e0 & 15) >> 2;       // code word of the block holding them
         const bool high = e0 >= 16;
         const int nt = min(kAttThreads, t1 - tb);
-        for (int j = warp; j < nt; j += 4) {
-            const int64_t r = head_row + tb + j;
-            const uint32_t w = __ldg(reinterpret_cast<const uint32_t *>(vc + r * (D / 2) + 16 * b) + word);
-            const float db = __half2float(__ushort_as_half(__ldg(vs + r * NB + b)));
-            float lo[4], hi[4];
-            nibbles(w, lo, hi);
+        // four tokens per step, their loads issued before any is used
+        constexpr int U = 4;
+        for (int j0 = warp; j0 < nt; j0 += 4 * U) {
+            uint32_t w[U];
+            float db[U];
 #pragma unroll
-            for (int h = 0; h < GQ; ++h) {
-                const float pd = p[h][j] * db;
+            for (int u = 0; u < U; ++u) {
+                const int j = j0 + 4 * u;
+                w[u] = 0;
+                db[u] = 0.0f;
+                if (j < nt) {
+                    const int64_t r = head_row + tb + j;
+                    w[u] = __ldg(reinterpret_cast<const uint32_t *>(vc + r * (D / 2) + 16 * b) + word);
+                    db[u] = __half2float(__ushort_as_half(__ldg(vs + r * NB + b)));
+                }
+            }
 #pragma unroll
-                for (int e = 0; e < 4; ++e) acc[h][e] = fmaf(pd, (high ? hi[e] : lo[e]) - 8.0f, acc[h][e]);
+            for (int u = 0; u < U; ++u) {
+                const int j = j0 + 4 * u;
+                if (j >= nt) break;
+                float lo[4], hi[4];
+                nibbles(w[u], lo, hi);
+#pragma unroll
+                for (int h = 0; h < GQ; ++h) {
+                    const float pd = p[h][j] * db[u];
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) acc[h][e] = fmaf(pd, (high ? hi[e] : lo[e]) - 8.0f, acc[h][e]);
+                }
             }
         }
         // exp-sum of the pass
@@ -254,9 +273,10 @@ cudaError_t launch_split(const float *q, int Hkv, int capacity, int L, int chunk
 }  // namespace
 
 int attention_chunk(int L, int Hkv, int num_sms) {
-    // enough CTAs for about two waves of the SMs, chunks of at least one pass
+    // chunks of whole passes, as many CTAs as about eight per SM hold at once
+    // (128 threads and under 32 KB of shared memory each)
     int chunk = kAttThreads;
-    while (static_cast<long long>((L + chunk - 1) / chunk) * Hkv > 2LL * num_sms && chunk < (1 << 20))
+    while (static_cast<long long>((L + chunk - 1) / chunk) * Hkv > 8LL * num_sms && chunk < (1 << 20))
         chunk *= 2;
     return chunk;
 }

@@ -18,9 +18,8 @@
 //    it streams its items into a ring of shared-memory slots: the 32 x 128 B
 //    code tile by TMA (128-byte swizzle, L2 evict-first, no multicast) and the
 //    unit's 32 x GPS scales, re-tiled at load time into unit order, by a bulk
-//    copy.  A CTA of the next kernel, resident beside this one under
-//    programmatic dependent launch, fills its own ring meanwhile.
-//  * Warps 1..8 are consumers.  The input is quantised once per cluster of C
+//    copy.
+//  * Warps 1..16 are consumers.  The input is quantised once per cluster of C
 //    CTAs: each CTA takes 1/C of the 128-blocks of the fp32 input, forms its
 //    share of max |x| (max |H x| with the Hadamard rotation) and of sum x^2,
 //    sends it to every CTA of the cluster (st.async into their shared
@@ -47,19 +46,26 @@
 namespace tern {
 namespace {
 
-constexpr int kSkConsumers = 8;
+constexpr int kSkConsumers = 16;
 constexpr int kSkThreads = 32 * (kSkConsumers + 1);
 constexpr int kSkBar = 1;   // named barrier of the consumer warps
 // Input blocks a consumer warp loads at once (one round) and keeps in
-// registers between the two passes: a K of 5 x 8 warps x 128 = 5120 per CTA
-// is one round; a longer share takes several, the earlier ones loaded again
-// for the second pass.  The prologue is unrolled over a round and runs once
-// per launch: rounds of 9 (one round up to K = 18432 with clusters of 2)
-// measured slower, their code costing more than the reloads they save.
+// registers between the two passes: a K of 5 x 16 warps x 128 = 10240 per
+// CTA is one round; a longer share takes several, the earlier ones loaded
+// again for the second pass.  The prologue is unrolled over a round and runs
+// once per launch: rounds of 9 measured slower (with 8 consumer warps), their
+// code costing more than the reloads they save.
 constexpr int kSkKeep = 5;
 constexpr int kSkMaxCluster = 4;
-constexpr int kSkSmemBudget = 112 * 1024;  // two CTAs per SM (programmatic launch overlap)
-constexpr int kSkMinRing = 8, kSkMaxRing = 24;  // unit slots, multiples of kSkChunk
+// One CTA per SM with 16 consumer warps and a ring of up to 40 unit slots.
+// Measured on B200 against two CTAs per SM with 8 consumer warps and a
+// 24-slot ring (which let the next launch's CTA prefetch beside this one):
+// 2.73 vs 3.05 ms per base-3 decode step, 2.34 vs 2.46 ms for 2-bit.  The
+// small projections (12 and 9 units per CTA) then decode every item at once
+// instead of two after another; 20 consumer warps spill, 24 or 48 slots
+// gain nothing.
+constexpr int kSkSmemBudget = 200 * 1024;
+constexpr int kSkMinRing = 8, kSkMaxRing = 40;  // unit slots, multiples of kSkChunk
 constexpr int kSkChunk = 4;                      // unit slots filled by one chunk of loads
 
 template <int FMT>
@@ -311,7 +317,7 @@ __device__ __forceinline__ int64_t tag_index(int rb, int mat, int m, int lane) {
 }
 
 template <int FMT, int MT, int MODE, bool DBG>
-__global__ void __launch_bounds__(kSkThreads, 2)
+__global__ void __launch_bounds__(kSkThreads, 1)
     gemv_stream_kernel(const __grid_constant__ CUtensorMap tm0,
                        const __grid_constant__ CUtensorMap tm1,
                        const __grid_constant__ CUtensorMap tm3_0,
@@ -860,10 +866,10 @@ cudaError_t launch_sk(const StreamLaunch &S, cudaStream_t s, const char **why) {
     e = once.run(dev, [&]() {
         cudaError_t r = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
         if (r != cudaSuccess) return r;
-        // Every launch takes the largest shared-memory split of the SM, so
-        // that a launch waiting on its predecessor (programmatic launch) can
-        // sit beside it on the same SM: launches whose splits differ cannot
-        // share an SM, which then drains before the next one starts.
+        // Every launch of the library takes the largest shared-memory split
+        // of the SM, so that consecutive launches never need the SM to be
+        // reconfigured (a split that differs from the previous launch's
+        // waits until the SM has drained).
         r = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout,
                                  cudaSharedmemCarveoutMaxShared);
         if (r != cudaSuccess) return r;
