@@ -49,24 +49,28 @@ namespace {
 constexpr int kGmTileN = 128;   // weight rows per CTA (MMA M)
 constexpr int kGmTile = 128 * 128;  // bytes of one 128 x 128 B int8 tile (codes, decoded A)
 constexpr int kGmCodeStages = 2;
-constexpr int kGmActStages = 3;
-constexpr int kGmAStages = 2;
 constexpr int kGmDecodeWarps = 4;
 constexpr int kGmEpiWarps = 16;
 constexpr int kGmWarps = 2 + kGmDecodeWarps + kGmEpiWarps;
 constexpr int kGmThreads = 32 * kGmWarps;
-constexpr int kGmAccBufs = 2;
 constexpr int kGmBand = 8;                     // weight-row tiles per raster band
 constexpr int kGmEpiBar = 1;                   // named barrier of the epilogue warps
 constexpr int kGmMaxSplit = 8;                 // portable cluster size
 
 // Sizes that follow from the token tile TM (MMA N): 64, 128 or 256 tokens.
+// The 64-token tile has little MMA and drain work per group: the time of a
+// group there is the latency of decode -> MMA -> drain, so it keeps four
+// groups in flight (activation tiles, decoded weight tiles, accumulators);
+// the wider tiles keep two or three.
 template <int TM>
 struct GmShape {
     static_assert(TM == 64 || TM == 128 || TM == 256, "token tile");
+    static constexpr int kActStages = TM == 64 ? 4 : 3;
+    static constexpr int kAStages = TM == 64 ? 4 : 2;
+    static constexpr int kAccBufs = TM == 64 ? 4 : 2;
     static constexpr int kActTile = TM * 128;          // one TM x 128 B activation tile
     static constexpr int kEpiCols = TM * 4 / kGmEpiWarps;  // token columns per epilogue warp
-    static constexpr int kTmemCols = TM * kGmAccBufs;  // accumulators (a power of two)
+    static constexpr int kTmemCols = TM * kAccBufs;    // accumulators (a power of two)
     static_assert(kTmemCols <= 512, "tensor memory holds 512 columns");
 };
 
@@ -82,12 +86,12 @@ struct GemmParams {
 template <int TM>
 struct GemmSmem {
     uint8_t code[kGmCodeStages][kGmTile];
-    uint8_t act[kGmActStages][GmShape<TM>::kActTile];
-    uint8_t a[kGmAStages][kGmTile];
+    uint8_t act[GmShape<TM>::kActStages][GmShape<TM>::kActTile];
+    uint8_t a[GmShape<TM>::kAStages][kGmTile];
     uint64_t code_full[kGmCodeStages], code_empty[kGmCodeStages];
-    uint64_t act_full[kGmActStages], act_empty[kGmActStages];
-    uint64_t a_full[kGmAStages], a_empty[kGmAStages];
-    uint64_t acc_full[kGmAccBufs], acc_empty[kGmAccBufs];
+    uint64_t act_full[GmShape<TM>::kActStages], act_empty[GmShape<TM>::kActStages];
+    uint64_t a_full[GmShape<TM>::kAStages], a_empty[GmShape<TM>::kAStages];
+    uint64_t acc_full[GmShape<TM>::kAccBufs], acc_empty[GmShape<TM>::kAccBufs];
     uint32_t tmem_base;
     // followed, with a split of K, by this rank's fp32 partial tile [TM][128]
     // (token-major), then by the tile's group scales, fp16 [GL][128]
@@ -143,6 +147,9 @@ __global__ void __launch_bounds__(kGmThreads, 1)
     using Sh = GmShape<TM>;
     constexpr int GPS = FMT == TERN_FMT_BASE3 ? 5 : 4;  // groups per superblock
     constexpr int EC = Sh::kEpiCols;
+    constexpr int kGmActStages = Sh::kActStages;
+    constexpr int kGmAStages = Sh::kAStages;
+    constexpr int kGmAccBufs = Sh::kAccBufs;
     extern __shared__ uint8_t smem_raw[];
     GemmSmem<TM> &S = *reinterpret_cast<GemmSmem<TM> *>(
         smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023));
