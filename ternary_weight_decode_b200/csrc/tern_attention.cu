@@ -15,11 +15,16 @@
 //    and a chunk of tokens and serves all Hq/Hkv query heads of that group,
 //    so each cached byte is read once per token.  Scores: a thread per token
 //    (its codes as four 16-byte loads), sum_b d_b (sum_i q_i c_i - 8 sum_i q_i)
-//    with the per-block query sums precomputed.  Values: a warp per token, a
-//    lane per four dimensions, p_t d_b (c - 8) accumulated in fp32.  The CTA
-//    writes its chunk's max score, exp-sum and unnormalised output.  Chunks
-//    are sized for about eight resident CTAs per SM, so the loads of many
-//    warps are in flight at once.
+//    with the per-block query sums precomputed.  Values: the pass's V rows
+//    copied into shared memory (cp.async) while the scores are formed, then
+//    a warp per token, a lane per four dimensions, p_t d_b (c - 8)
+//    accumulated in fp32.  The CTA
+//    writes its chunk's max score, exp-sum and unnormalised output.  The
+//    codes become floats as the bits of 2^23 + c less 2^23 (no conversion
+//    instruction); one thread starts a bulk L2 prefetch of the K and V rows
+//    two passes ahead, so each pass's loads find them in L2.  Chunks are
+//    sized from the CTAs an SM holds at once so that the grid fills whole
+//    waves of the SMs.
 //  * attn_combine_kernel: per query head, the chunks' partial results merged
 //    in chunk order with the running-max rule (a fixed order: the result
 //    does not depend on timing).
@@ -60,31 +65,89 @@ __global__ void kv_append_kernel(const float *__restrict__ x, int H, int D, int 
     scales[row * nb + b] = __half_as_ushort(__float2half_rn(d));
 }
 
+// Codes as floats without the conversion unit: byte e of `nib` (a nibble,
+// 0..15) becomes the low byte of the bit pattern of 2^23 + c, from which
+// one subtraction leaves c - bias exactly (every value here is an integer
+// below 2^24, where one ulp is 1).
+constexpr uint32_t kNibMagic = 0x4B000000u;  // 2^23 as fp32 bits
+__device__ __forceinline__ float nib_float(uint32_t nib, int e, float bias) {
+    return __fsub_rn(__uint_as_float(__byte_perm(nib, kNibMagic, 0x7640 + e)), 8388608.0f + bias);
+}
+
 // Nibble values of a 32-bit word as floats: lo[e] = byte e & 15, hi[e] = byte e >> 4.
 __device__ __forceinline__ void nibbles(uint32_t w, float (&lo)[4], float (&hi)[4]) {
+    const uint32_t l = w & 0x0F0F0F0Fu, h = (w >> 4) & 0x0F0F0F0Fu;
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
-        lo[e] = static_cast<float>((w >> (8 * e)) & 15u);
-        hi[e] = static_cast<float>((w >> (8 * e + 4)) & 15u);
+        lo[e] = nib_float(l, e, 0.0f);
+        hi[e] = nib_float(h, e, 0.0f);
     }
 }
+
+// Bulk prefetch into L2 (no shared memory, no completion): `bytes` from a
+// 16-byte aligned address, a multiple of 16.
+__device__ __forceinline__ void prefetch_l2(const void *p, uint32_t bytes) {
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(reinterpret_cast<uint64_t>(p)), "r"(bytes)
+                 : "memory");
+}
+
+// The K and V rows (codes, and scales when `scales16`: both scale arrays
+// 16-byte aligned) of tokens [t, t + n) of one head, into L2.  Scale rows
+// are 8 bytes: the range is shrunk to whole 16-byte pairs inside it.
+__device__ __forceinline__ void prefetch_rows(int64_t row, int n, const uint8_t *kc, const uint16_t *ks,
+                                              const uint8_t *vc, const uint16_t *vs, bool scales16) {
+    if (n <= 0) return;
+    prefetch_l2(kc + row * (kAttD / 2), static_cast<uint32_t>(n) * (kAttD / 2));
+    prefetch_l2(vc + row * (kAttD / 2), static_cast<uint32_t>(n) * (kAttD / 2));
+    const int64_t r0 = (row + 1) & ~static_cast<int64_t>(1), r1 = (row + n) & ~static_cast<int64_t>(1);
+    if (scales16 && r1 > r0) {
+        constexpr int NB = kAttD / 32;
+        prefetch_l2(ks + r0 * NB, static_cast<uint32_t>(r1 - r0) * NB * 2);
+        prefetch_l2(vs + r0 * NB, static_cast<uint32_t>(r1 - r0) * NB * 2);
+    }
+}
+
+// Asynchronous copies global -> shared (no registers held while in flight).
+__device__ __forceinline__ void cp_async16(void *dst, const void *src) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst)),
+                 "l"(reinterpret_cast<uint64_t>(src))
+                 : "memory");
+}
+__device__ __forceinline__ void cp_async8(void *dst, const void *src) {
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 8;" ::"r"(smem_u32(dst)),
+                 "l"(reinterpret_cast<uint64_t>(src))
+                 : "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
+
+// Launch flags of the split kernel: alignment of the scale arrays.
+constexpr int kScales16 = 1;  // both scale arrays 16-byte aligned (L2 prefetch of scales)
+constexpr int kVScales8 = 2;  // v_scales 8-byte aligned (one 8-byte copy per token)
 
 template <int GQ>
 __global__ void __launch_bounds__(kAttThreads)
     attn_split_kernel(const float *__restrict__ q, int Hkv, int capacity, int L, int chunk,
                       const uint8_t *__restrict__ kc, const uint16_t *__restrict__ ks,
                       const uint8_t *__restrict__ vc, const uint16_t *__restrict__ vs,
-                      float *__restrict__ part, int nchunks) {
+                      float *__restrict__ part, int nchunks, int flags) {
     constexpr int D = kAttD, NB = D / 32;
     __shared__ __align__(16) float qs[GQ][D];  // the group's queries
     __shared__ float qsum[GQ][NB];       // sum of q over each block of 32
     __shared__ float p[GQ][kAttThreads]; // scores, then exp(score - max), of one pass
     __shared__ float red[GQ][4][D];      // the warps' partial outputs
     __shared__ float wmax[GQ][4], wsum[GQ][4];
+    __shared__ __align__(16) uint8_t vt[kAttThreads][D / 2];  // the pass's V codes
+    __shared__ __align__(16) uint16_t vst[kAttThreads][NB];   // and their block scales
+    const bool scales16 = (flags & kScales16) != 0;
     const int g = blockIdx.y, ck = blockIdx.x;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int t0 = ck * chunk, t1 = min(L, t0 + chunk);
     const float inv_sqrt_d = 0.08838834764831845f;  // 1/sqrt(128) rounded to fp32
+    const int64_t head_row = static_cast<int64_t>(g) * capacity;
+    // The first two passes' rows start towards L2 before the wait (L2 is
+    // coherent: the token the previous kernel appends is read after it).
+    if (tid == 0)
+        prefetch_rows(head_row + t0, min(2 * kAttThreads, t1 - t0), kc, ks, vc, vs, scales16);
     pdl_wait();  // q (and the appended token) come from earlier kernels
     for (int i = tid; i < GQ * D; i += kAttThreads) (&qs[0][0])[i] = q[static_cast<int64_t>(g) * GQ * D + i];
     __syncthreads();
@@ -103,10 +166,28 @@ __global__ void __launch_bounds__(kAttThreads)
         for (int e = 0; e < 4; ++e) acc[h][e] = 0.0f;
     }
     __syncthreads();
-    const int64_t head_row = static_cast<int64_t>(g) * capacity;
-    // passes of kAttThreads tokens: scores, then the value accumulation
+    // passes of kAttThreads tokens: scores, then the value accumulation;
+    // the pass two ahead is prefetched into L2 as each one starts
     for (int tb = t0; tb < t1; tb += kAttThreads) {
         const int t = tb + tid;
+        if (tid == 0) {
+            const int tp = tb + 2 * kAttThreads;
+            prefetch_rows(head_row + tp, min(kAttThreads, t1 - tp), kc, ks, vc, vs, scales16);
+        }
+        const int nt = min(kAttThreads, t1 - tb);
+        // this pass's V rows into shared memory, in flight while the scores
+        // are formed (the previous pass's readers are past its last barrier)
+        for (int i = tid; i < nt * 4; i += kAttThreads)
+            cp_async16(&vt[i >> 2][16 * (i & 3)], vc + (head_row + tb + (i >> 2)) * (D / 2) + 16 * (i & 3));
+        if (tid < nt) {
+            const uint16_t *src = vs + (head_row + tb + tid) * NB;
+            if (flags & kVScales8) {
+                cp_async8(&vst[tid][0], src);
+            } else {
+#pragma unroll
+                for (int b = 0; b < NB; ++b) vst[tid][b] = __ldg(src + b);
+            }
+        }
         float sc[GQ];
         if (t < t1) {
             const uint4 *krow = reinterpret_cast<const uint4 *>(kc + (head_row + t) * (D / 2));
@@ -170,14 +251,14 @@ __global__ void __launch_bounds__(kAttThreads)
             m_run[h] = mn;
             p[h][tid] = t < t1 ? expf(sc[h] - mn) : 0.0f;
         }
+        cp_async_wait_all();  // this thread's V copies have landed
         __syncthreads();
         // values: warp w takes tokens w, w+4, ... of the pass; lane = dims 4l..4l+3
         const int b = lane >> 3;               // block of the lane's dims
         const int e0 = (4 * lane) & 31;        // first element inside the block
         const int word = (e0 & 15) >> 2;       // code word of the block holding them
         const bool high = e0 >= 16;
-        const int nt = min(kAttThreads, t1 - tb);
-        // four tokens per step, their loads issued before any is used
+        // four tokens per step, from shared memory
         constexpr int U = 4;
         for (int j0 = warp; j0 < nt; j0 += 4 * U) {
             uint32_t w[U];
@@ -188,22 +269,24 @@ __global__ void __launch_bounds__(kAttThreads)
                 w[u] = 0;
                 db[u] = 0.0f;
                 if (j < nt) {
-                    const int64_t r = head_row + tb + j;
-                    w[u] = __ldg(reinterpret_cast<const uint32_t *>(vc + r * (D / 2) + 16 * b) + word);
-                    db[u] = __half2float(__ushort_as_half(__ldg(vs + r * NB + b)));
+                    w[u] = *reinterpret_cast<const uint32_t *>(&vt[j][16 * b + 4 * word]);
+                    db[u] = __half2float(__ushort_as_half(vst[j][b]));
                 }
             }
 #pragma unroll
             for (int u = 0; u < U; ++u) {
                 const int j = j0 + 4 * u;
                 if (j >= nt) break;
-                float lo[4], hi[4];
-                nibbles(w[u], lo, hi);
+                // only the lane's four nibbles, as c - 8
+                const uint32_t nib = (w[u] >> (high ? 4 : 0)) & 0x0F0F0F0Fu;
+                float cv[4];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) cv[e] = nib_float(nib, e, 8.0f);
 #pragma unroll
                 for (int h = 0; h < GQ; ++h) {
                     const float pd = p[h][j] * db[u];
 #pragma unroll
-                    for (int e = 0; e < 4; ++e) acc[h][e] = fmaf(pd, (high ? hi[e] : lo[e]) - 8.0f, acc[h][e]);
+                    for (int e = 0; e < 4; ++e) acc[h][e] = fmaf(pd, cv[e], acc[h][e]);
                 }
             }
         }
@@ -266,23 +349,56 @@ cudaError_t launch_split(const float *q, int Hkv, int capacity, int L, int chunk
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
+    const auto ks = reinterpret_cast<uintptr_t>(C.k_scales), vs = reinterpret_cast<uintptr_t>(C.v_scales);
+    const int flags = (ks % 16 == 0 && vs % 16 == 0 ? kScales16 : 0) | (vs % 8 == 0 ? kVScales8 : 0);
     return cudaLaunchKernelEx(&cfg, attn_split_kernel<GQ>, q, Hkv, capacity, L, chunk, C.k_codes,
-                              C.k_scales, C.v_codes, C.v_scales, part, nchunks);
+                              C.k_scales, C.v_codes, C.v_scales, part, nchunks, flags);
+}
+
+// Split CTAs one SM holds at once (registers and shared memory of the
+// instantiation for GQ query heads per KV head); 1 for an unsupported GQ.
+int split_ctas_per_sm(int GQ) {
+    const void *k = nullptr;
+    switch (GQ) {
+        case 1: k = reinterpret_cast<const void *>(attn_split_kernel<1>); break;
+        case 2: k = reinterpret_cast<const void *>(attn_split_kernel<2>); break;
+        case 4: k = reinterpret_cast<const void *>(attn_split_kernel<4>); break;
+        case 5: k = reinterpret_cast<const void *>(attn_split_kernel<5>); break;
+        case 8: k = reinterpret_cast<const void *>(attn_split_kernel<8>); break;
+        default: return 1;
+    }
+    int n = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, k, kAttThreads, 0) != cudaSuccess || n < 1) {
+        (void)cudaGetLastError();
+        return 1;
+    }
+    return n;
 }
 
 }  // namespace
 
-int attention_chunk(int L, int Hkv, int num_sms) {
-    // chunks of whole passes, as many CTAs as about eight per SM hold at once
-    // (128 threads and under 32 KB of shared memory each)
-    int chunk = kAttThreads;
-    while (static_cast<long long>((L + chunk - 1) / chunk) * Hkv > 8LL * num_sms && chunk < (1 << 20))
-        chunk *= 2;
-    return chunk;
+int attention_chunk(int L, int Hkv, int GQ, int num_sms) {
+    // Chunks of whole passes, chosen so that the CTAs fill whole waves of
+    // the SMs: the least tokens that one resident CTA slot has to stream
+    // (waves x chunk), the fewer CTAs on a tie.
+    const long long slots = static_cast<long long>(split_ctas_per_sm(GQ)) * num_sms;
+    long long best = kAttThreads, best_cost = -1;
+    for (long long w = 1; w <= 64; ++w) {
+        const long long per_head = w * slots / Hkv > 0 ? w * slots / Hkv : 1;
+        long long chunk = (L + per_head - 1) / per_head;
+        chunk = (chunk + kAttThreads - 1) / kAttThreads * kAttThreads;
+        const long long ctas = (L + chunk - 1) / chunk * Hkv;
+        const long long cost = (ctas + slots - 1) / slots * chunk;
+        if (best_cost < 0 || cost < best_cost || (cost == best_cost && chunk > best)) {
+            best = chunk;
+            best_cost = cost;
+        }
+    }
+    return static_cast<int>(best);
 }
 
 size_t attention_workspace_bytes(int Hq, int L, int Hkv, int num_sms) {
-    const int chunk = attention_chunk(L, Hkv, num_sms);
+    const int chunk = attention_chunk(L, Hkv, Hq / Hkv, num_sms);
     const size_t nchunks = static_cast<size_t>((L + chunk - 1) / chunk);
     return static_cast<size_t>(Hq) * nchunks * (kAttD + 2) * sizeof(float);
 }
@@ -300,7 +416,7 @@ cudaError_t launch_kv_append(const float *k, const float *v, int pos, const tern
 cudaError_t launch_attention(const float *q, int Hq, const tern_kv_cache &C, int L, float *out,
                              float *part, int num_sms, cudaStream_t s, const char **why) {
     const int GQ = Hq / C.Hkv;
-    const int chunk = attention_chunk(L, C.Hkv, num_sms);
+    const int chunk = attention_chunk(L, C.Hkv, GQ, num_sms);
     const int nchunks = (L + chunk - 1) / chunk;
     cudaError_t e;
     switch (GQ) {

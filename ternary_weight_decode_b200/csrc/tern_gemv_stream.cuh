@@ -150,19 +150,24 @@ template <int FMT, int MT, typename Words4, typename Sink>
 __device__ __forceinline__ void sk_item(Words4 words4, const float (&sc)[Fmt<FMT>::kGroups],
                                         const uint8_t *act_sb, int Kpad, const int *sq_sb, int GT,
                                         float (&yacc)[MT], Sink sink) {
-    int acc[MT];
+    // Two integer chains (base-3: even and odd digit words), so that one
+    // dp4a need not wait for the one before; their sum is exact.
+    int acc[MT], acc2[MT];
 #pragma unroll
     for (int m = 0; m < MT; ++m) {
         acc[m] = 0;
+        acc2[m] = 0;
         yacc[m] = 0.0f;
     }
     // sum w q = sum t q - sum q over the group (t = w + 1); the bit-plane
     // path accumulates sum w q itself
     auto finish = [&](int m, int g) {
-        const int P = FMT == TERN_FMT_BITPLANE ? acc[m] : acc[m] - sq_sb[(m * GT + g) * 4];
+        const int S = acc[m] + acc2[m];
+        const int P = FMT == TERN_FMT_BITPLANE ? S : S - sq_sb[(m * GT + g) * 4];
         sink(m, g, P);
         yacc[m] = fmaf(sc[g], static_cast<float>(P), yacc[m]);
         acc[m] = 0;
+        acc2[m] = 0;
     };
 #pragma unroll
     for (int c = 0; c < 8; ++c) {
@@ -193,7 +198,10 @@ __device__ __forceinline__ void sk_item(Words4 words4, const float (&sc)[Fmt<FMT
                 for (int d = 0; d < 20; ++d) {
                     const int dd = c * 20 + d;
                     if (dd > 0 && (dd & 31) == 0) finish(m, (dd >> 5) - 1);
-                    acc[m] = dp4a_ss(t[d], aw[d], acc[m]);
+                    if (d & 1)
+                        acc2[m] = dp4a_ss(t[d], aw[d], acc2[m]);
+                    else
+                        acc[m] = dp4a_ss(t[d], aw[d], acc[m]);
                 }
             }
         } else if constexpr (FMT == TERN_FMT_BITPLANE) {
@@ -522,17 +530,20 @@ __global__ void __launch_bounds__(kSkThreads, 1)
             }
         }
         warpgroup_sync_n(kSkBar, kSkConsumers * 32);
-        // This CTA's share, combined by every thread in the same warp order.
+        // This CTA's share: lane w holds warp w's, combined across the lanes
+        // by the same butterfly in every warp (hence the same sum in every
+        // lane, warp and CTA).
+        static_assert(kSkConsumers <= 32, "one consumer warp per lane");
         float amax_c[MT], ss_c[MT];
 #pragma unroll
         for (int m = 0; m < MT; ++m) {
             float a = 0.0f, s = 0.0f;
-            for (int w = 0; w < kSkConsumers; ++w) {
-                a = fmaxf(a, red[(w * MT + m) * 2 + 0]);
-                s += red[(w * MT + m) * 2 + 1];
+            if (lane < kSkConsumers) {
+                a = red[(lane * MT + m) * 2 + 0];
+                s = red[(lane * MT + m) * 2 + 1];
             }
-            amax_c[m] = a;
-            ss_c[m] = s;
+            amax_c[m] = __uint_as_float(__reduce_max_sync(0xffffffffu, __float_as_uint(a)));
+            ss_c[m] = warp_sum(s);
         }
         bool ok1 = true;
         if (C > 1) {

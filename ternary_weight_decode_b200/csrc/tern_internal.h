@@ -86,7 +86,7 @@ cudaError_t launch_ternarize(const float *w, int N, int K, int ldw, int8_t *trit
 // ---------------------------------------------------------------- attention
 cudaError_t launch_kv_append(const float *k, const float *v, int pos, const tern_kv_cache &C,
                              cudaStream_t s);
-int attention_chunk(int L, int Hkv, int num_sms);
+int attention_chunk(int L, int Hkv, int GQ, int num_sms);
 size_t attention_workspace_bytes(int Hq, int L, int Hkv, int num_sms);
 cudaError_t launch_attention(const float *q, int Hq, const tern_kv_cache &C, int L, float *out,
                              float *part, int num_sms, cudaStream_t s, const char **why);
