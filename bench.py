@@ -22,6 +22,7 @@ each with a bounded sample of the CPU oracle timed on this host.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
                     [--fmt base3|2bit] [--layers 64] [--M 1] [--quick]
+    python bench.py --attention 4096 65536      # c7 alone
 
 N > 1 runs N independent replicas (one process per GPU, launched by
 torch.distributed.run): the path has no cross-GPU exchange step.
@@ -64,6 +65,9 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-prefill", action="store_true", help="skip the prefill GEMM (c5)")
     ap.add_argument("--quick", action="store_true", help="headline step only (no c1..c5)")
+    ap.add_argument("--attention", type=int, nargs="+", default=None, metavar="L",
+                    help="decode attention (c7) alone at these context lengths, one GPU; "
+                         "prints its JSON and no decode step")
     return ap.parse_args()
 
 
@@ -724,6 +728,11 @@ def main():
     from ternary_weight_decode_b200 import decode, synth, tern
 
     torch.cuda.set_device(local)
+    if args.attention:
+        if world > 1:
+            raise SystemExit("--attention runs on one GPU")
+        print(json.dumps({"config": "c7_attention", **attention_sweep(Ls=tuple(args.attention))}))
+        return 0
     fmt_id = fmt_id_of(args.fmt)
     mode = args.mode if args.mode != "auto" else ("streamed" if args.M <= 2 else "fused")
     model = decode.DecodeModel(fmt_id, args.layers, M=args.M, mode=mode).build(seed_base=0)
