@@ -26,8 +26,9 @@
 //    sized from the CTAs an SM holds at once so that the grid fills whole
 //    waves of the SMs.
 //  * attn_combine_kernel: per query head, the chunks' partial results merged
-//    in chunk order with the running-max rule (a fixed order: the result
-//    does not depend on timing).
+//    with the running-max rule: the chunk weights once in shared memory,
+//    then four chunk lanes per dimension, each in chunk order, added in lane
+//    order (a fixed order: the result does not depend on timing).
 #include "tern_common.cuh"
 #include "tern_internal.h"
 
@@ -36,7 +37,7 @@ namespace {
 
 constexpr int kAttD = 128;         // head dimension
 constexpr int kAttThreads = 128;   // 4 warps
-constexpr int kAttMaxGroup = 8;    // query heads per KV head
+constexpr int kAttMaxChunks = 8192;  // chunks of the context per KV head
 
 __global__ void kv_append_kernel(const float *__restrict__ x, int H, int D, int pos, int capacity,
                                  uint8_t *__restrict__ codes, uint16_t *__restrict__ scales) {
@@ -157,13 +158,14 @@ __global__ void __launch_bounds__(kAttThreads)
         for (int i = 0; i < 32; ++i) s += qs[h][32 * b + i];
         qsum[h][b] = s;
     }
-    float m_run[GQ], z_run[GQ], acc[GQ][4];
+    float m_run[GQ], z_run[GQ];
+    float2 acc[GQ][2];  // the lane's four dimensions, two per packed instruction
 #pragma unroll
     for (int h = 0; h < GQ; ++h) {
         m_run[h] = -INFINITY;
         z_run[h] = 0.0f;
 #pragma unroll
-        for (int e = 0; e < 4; ++e) acc[h][e] = 0.0f;
+        for (int e = 0; e < 2; ++e) acc[h][e] = make_float2(0.0f, 0.0f);
     }
     __syncthreads();
     // passes of kAttThreads tokens: scores, then the value accumulation;
@@ -198,9 +200,10 @@ __global__ void __launch_bounds__(kAttThreads)
             for (int b = 0; b < NB; ++b) {
                 const uint4 w = __ldg(krow + b);
                 const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
-                float dot[GQ];
+                // per head, even and odd elements in the two halves of a packed pair
+                float2 dot[GQ];
 #pragma unroll
-                for (int h = 0; h < GQ; ++h) dot[h] = 0.0f;
+                for (int h = 0; h < GQ; ++h) dot[h] = make_float2(0.0f, 0.0f);
 #pragma unroll
                 for (int c = 0; c < 4; ++c) {
                     float lo[4], hi[4];
@@ -210,21 +213,18 @@ __global__ void __launch_bounds__(kAttThreads)
                         // elements 4c..4c+3 (low nibbles) and 16+4c.. (high nibbles)
                         const float4 ql = *reinterpret_cast<const float4 *>(&qs[h][32 * b + 4 * c]);
                         const float4 qh = *reinterpret_cast<const float4 *>(&qs[h][32 * b + 16 + 4 * c]);
-                        float d = dot[h];
-                        d = fmaf(ql.x, lo[0], d);
-                        d = fmaf(ql.y, lo[1], d);
-                        d = fmaf(ql.z, lo[2], d);
-                        d = fmaf(ql.w, lo[3], d);
-                        d = fmaf(qh.x, hi[0], d);
-                        d = fmaf(qh.y, hi[1], d);
-                        d = fmaf(qh.z, hi[2], d);
-                        d = fmaf(qh.w, hi[3], d);
+                        float2 d = dot[h];
+                        d = __ffma2_rn(make_float2(ql.x, ql.y), make_float2(lo[0], lo[1]), d);
+                        d = __ffma2_rn(make_float2(ql.z, ql.w), make_float2(lo[2], lo[3]), d);
+                        d = __ffma2_rn(make_float2(qh.x, qh.y), make_float2(hi[0], hi[1]), d);
+                        d = __ffma2_rn(make_float2(qh.z, qh.w), make_float2(hi[2], hi[3]), d);
                         dot[h] = d;
                     }
                 }
                 const float db = __half2float(__ushort_as_half(__ldg(kd + b)));
 #pragma unroll
-                for (int h = 0; h < GQ; ++h) sc[h] = fmaf(db, fmaf(-8.0f, qsum[h][b], dot[h]), sc[h]);
+                for (int h = 0; h < GQ; ++h)
+                    sc[h] = fmaf(db, fmaf(-8.0f, qsum[h][b], dot[h].x + dot[h].y), sc[h]);
             }
 #pragma unroll
             for (int h = 0; h < GQ; ++h) sc[h] *= inv_sqrt_d;
@@ -247,7 +247,7 @@ __global__ void __launch_bounds__(kAttThreads)
             const float r = m_run[h] == -INFINITY ? 0.0f : expf(m_run[h] - mn);
             z_run[h] *= r;
 #pragma unroll
-            for (int e = 0; e < 4; ++e) acc[h][e] *= r;
+            for (int e = 0; e < 2; ++e) acc[h][e] = make_float2(acc[h][e].x * r, acc[h][e].y * r);
             m_run[h] = mn;
             p[h][tid] = t < t1 ? expf(sc[h] - mn) : 0.0f;
         }
@@ -286,7 +286,8 @@ __global__ void __launch_bounds__(kAttThreads)
                 for (int h = 0; h < GQ; ++h) {
                     const float pd = p[h][j] * db[u];
 #pragma unroll
-                    for (int e = 0; e < 4; ++e) acc[h][e] = fmaf(pd, cv[e], acc[h][e]);
+                    for (int e = 0; e < 2; ++e)
+                        acc[h][e] = __ffma2_rn(make_float2(pd, pd), make_float2(cv[2 * e], cv[2 * e + 1]), acc[h][e]);
                 }
             }
         }
@@ -304,7 +305,7 @@ __global__ void __launch_bounds__(kAttThreads)
 #pragma unroll
     for (int h = 0; h < GQ; ++h)
 #pragma unroll
-        for (int e = 0; e < 4; ++e) red[h][warp][4 * lane + e] = acc[h][e];
+        for (int e = 0; e < 4; ++e) red[h][warp][4 * lane + e] = (e & 1) ? acc[h][e >> 1].y : acc[h][e >> 1].x;
     __syncthreads();
     for (int i = tid; i < GQ * D; i += kAttThreads) {
         const int h = i / D, d = i % D;
@@ -319,22 +320,56 @@ __global__ void __launch_bounds__(kAttThreads)
     pdl_launch_dependents();
 }
 
-__global__ void attn_combine_kernel(const float *__restrict__ part, int nchunks, float *__restrict__ out) {
+// Merge of one query head's chunk records: lane j of dimension d (S lanes
+// per dimension) sums chunks j, j + S, ... in order; the S partial sums are
+// added in lane order, so the result does not depend on timing.  The chunk
+// weights exp(m_c - M) are formed once, in shared memory.
+constexpr int kCombSplit = 4;
+constexpr int kCombThreads = kAttD * kCombSplit;
+
+__global__ void __launch_bounds__(kCombThreads)
+    attn_combine_kernel(const float *__restrict__ part, int nchunks, float *__restrict__ out) {
     constexpr int D = kAttD;
-    const int h = blockIdx.x, d = threadIdx.x;
+    extern __shared__ float wch[];  // [nchunks] chunk weights
+    __shared__ float wmax[kCombThreads / 32];
+    __shared__ float pnum[kCombSplit][D], pden[kCombSplit][D];
+    const int h = blockIdx.x, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int d = tid % D, j = tid / D;
     pdl_wait();
     const float *base = part + static_cast<int64_t>(h) * nchunks * (D + 2);
+    float m = -INFINITY;
+    for (int c = tid; c < nchunks; c += kCombThreads) m = fmaxf(m, base[c * (D + 2) + D]);
+    m = warp_max(m);
+    if (lane == 0) wmax[warp] = m;
+    __syncthreads();
     float M = -INFINITY;
-    for (int c = 0; c < nchunks; ++c) M = fmaxf(M, base[c * (D + 2) + D]);
+#pragma unroll
+    for (int w = 0; w < kCombThreads / 32; ++w) M = fmaxf(M, wmax[w]);
+    for (int c = tid; c < nchunks; c += kCombThreads) {
+        const float mc = base[c * (D + 2) + D];
+        wch[c] = mc == -INFINITY ? 0.0f : expf(mc - M);  // an empty chunk weighs nothing
+    }
+    __syncthreads();
     float num = 0.0f, den = 0.0f;
-    for (int c = 0; c < nchunks; ++c) {
+#pragma unroll 4
+    for (int c = j; c < nchunks; c += kCombSplit) {
         const float *rec = base + c * (D + 2);
-        if (rec[D] == -INFINITY) continue;  // an empty chunk
-        const float w = expf(rec[D] - M);
+        const float w = wch[c];
         num = fmaf(w, rec[d], num);
         den = fmaf(w, rec[D + 1], den);
     }
-    out[static_cast<int64_t>(h) * D + d] = num / den;
+    pnum[j][d] = num;
+    pden[j][d] = den;
+    __syncthreads();
+    if (j == 0) {
+        float n = pnum[0][d], z = pden[0][d];
+#pragma unroll
+        for (int i = 1; i < kCombSplit; ++i) {
+            n += pnum[i][d];
+            z += pden[i][d];
+        }
+        out[static_cast<int64_t>(h) * D + d] = n / z;
+    }
 }
 
 template <int GQ>
@@ -381,12 +416,15 @@ int attention_chunk(int L, int Hkv, int GQ, int num_sms) {
     // Chunks of whole passes, chosen so that the CTAs fill whole waves of
     // the SMs: the least tokens that one resident CTA slot has to stream
     // (waves x chunk), the fewer CTAs on a tie.
+    // At most kAttMaxChunks chunks (the merge keeps one weight per chunk in
+    // shared memory).
     const long long slots = static_cast<long long>(split_ctas_per_sm(GQ)) * num_sms;
-    long long best = kAttThreads, best_cost = -1;
+    auto whole_passes = [](long long t) { return (t + kAttThreads - 1) / kAttThreads * kAttThreads; };
+    long long best = whole_passes((L + kAttMaxChunks - 1) / kAttMaxChunks), best_cost = -1;
     for (long long w = 1; w <= 64; ++w) {
         const long long per_head = w * slots / Hkv > 0 ? w * slots / Hkv : 1;
-        long long chunk = (L + per_head - 1) / per_head;
-        chunk = (chunk + kAttThreads - 1) / kAttThreads * kAttThreads;
+        const long long chunk = whole_passes((L + per_head - 1) / per_head);
+        if ((L + chunk - 1) / chunk > kAttMaxChunks) continue;
         const long long ctas = (L + chunk - 1) / chunk * Hkv;
         const long long cost = (ctas + slots - 1) / slots * chunk;
         if (best_cost < 0 || cost < best_cost || (cost == best_cost && chunk > best)) {
@@ -430,7 +468,8 @@ cudaError_t launch_attention(const float *q, int Hq, const tern_kv_cache &C, int
     if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(Hq, 1, 1);
-    cfg.blockDim = dim3(kAttD, 1, 1);
+    cfg.blockDim = dim3(kCombThreads, 1, 1);
+    cfg.dynamicSmemBytes = static_cast<size_t>(nchunks) * sizeof(float);
     cfg.stream = s;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
