@@ -629,7 +629,7 @@ __global__ void __launch_bounds__(kSkThreads, 1)
                     quant_block(m, b, v[m][j]);
                 }
         }
-        fence_proxy_async_smem();  // the share is read by the bulk copies
+        if (C > 1) fence_proxy_async_smem();  // the share is read by the bulk copies
         warpgroup_sync_n(kSkBar, kSkConsumers * 32);
         if (ctid == 0 && nown > 0) {
             for (int q = 0; q < C; ++q) {
@@ -753,6 +753,19 @@ __global__ void __launch_bounds__(kSkThreads, 1)
                 }
             }
         }
+        // The warp that finishes the cut last row block reads the partial its
+        // neighbour published before the barrier, so that the load's latency
+        // overlaps the wait for the slowest warp; if the tag is not there yet
+        // it waits below.  (Every tag seen after the dependency wait is this
+        // launch's: each launch clears the words it used before it ends.)
+        unsigned long long early[NMAT][MT];
+        const bool combine_here = combine && (rb_hi - rb_lo) % kSkConsumers == cw && !(rb_hi == rb_lo && publish);
+#pragma unroll
+        for (int mat = 0; mat < NMAT; ++mat)
+#pragma unroll
+            for (int m = 0; m < MT; ++m)
+                early[mat][m] = combine_here ? ld_relaxed_gpu_u64(p.ws_tag + tag_index<NMAT, MT>(rb_hi, mat, m, lane))
+                                             : 0ull;
         warpgroup_sync_n(kSkBar, kSkConsumers * 32);
 
         // row blocks of this range: sum units in order; finish
@@ -779,7 +792,8 @@ __global__ void __launch_bounds__(kSkThreads, 1)
 #pragma unroll
                     for (int m = 0; m < MT; ++m) {
                         unsigned long long *t = p.ws_tag + tag_index<NMAT, MT>(rb, mat, m, lane);
-                        const unsigned long long w = wait_tagged_word(t);
+                        const unsigned long long w =
+                            (early[mat][m] >> 32) != 0 ? early[mat][m] : wait_tagged_word(t);
                         tot[mat][m] = tot[mat][m] + __uint_as_float(static_cast<uint32_t>(w));
                         st_relaxed_gpu_u64(t, 0ull);
                     }
