@@ -83,8 +83,8 @@ __device__ __forceinline__ uint32_t times3(uint32_t z) {
 }
 
 __device__ __forceinline__ void decode_d3_D(uint32_t X, uint32_t (&D)[5]) {
-    uint32_t ze = X & 0x00FF00FFu;         // bytes 0 and 2
-    uint32_t zo = (X >> 8) & 0x00FF00FFu;  // bytes 1 and 3
+    uint32_t ze = X & 0x00FF00FFu;              // bytes 0 and 2
+    uint32_t zo = __byte_perm(X, 0u, 0x4341);  // bytes 1 and 3: one permute, not a shift and a mask
 #pragma unroll
     for (int i = 0; i < 5; ++i) {
         ze = times3(ze);
