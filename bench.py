@@ -566,11 +566,12 @@ def ffn_sweep(model, fmt, peak, Ms=(1, 2, 4, 8, 16)):
             "faster_kernels_by_M": {str(M): r["kernels"] for M, r in sorted(best.items())}}
 
 
-def verify_sweep(model, fmt, Ms=(16, 32, 64, 128)):
+def verify_sweep(model, fmt, Ms=(4, 8, 16, 32, 64, 128)):
     """c6: multi-token verify on the tensor cores -- tern_gemm of the gate
     (K = 5120, N = 17408) and down (K = 17408, N = 5120) matrices of
     ROT_COPIES layers (weights never in L2) at M token rows (64- or
-    128-token tiles, a cluster split of K for down)."""
+    128-token tiles, a cluster split of K for down).  M = 4 and 8 place the
+    crossover with the CUDA-core kernels of c4 (GB/s of weights)."""
     import torch
     from ternary_weight_decode_b200 import tern
     L8 = model.layers[:ROT_COPIES]

@@ -931,7 +931,8 @@ cudaError_t launch_sk(const StreamLaunch &S, cudaStream_t s, const char **why) {
     while (C > 1 && want < C) C /= 2;
     p.nCTA = static_cast<int>((want / C) * C);
     const int items_max = sk_items_max<NMAT>(p.U, p.nCTA);
-    // ring depth: as many whole chunks as fit the two-CTAs-per-SM budget
+    // ring depth: as many whole chunks as fit the shared-memory budget of
+    // one CTA per SM
     int R = kSkMaxRing;
     while (R > kSkMinRing && sk_layout<FMT, MT>(p.SB, items_max, R).total > kSkSmemBudget)
         R -= kSkChunk;
