@@ -81,6 +81,17 @@ __device__ __forceinline__ void fence_proxy_async_smem() {
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
+// A warp hands a TMA-filled shared-memory buffer back to its producer: each
+// lane's reads of it (generic proxy) are ordered before the producer's next
+// TMA write into it (async proxy) by a proxy fence, then one arrival on the
+// buffer's empty barrier for the whole warp.  Without the fence the refill
+// may land before a lane's read of the old contents.
+__device__ __forceinline__ void release_to_tma(uint64_t *empty_bar, int lane) {
+    fence_proxy_async_smem();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(empty_bar);
+}
+
 __device__ __forceinline__ void prefetch_tmap(const CUtensorMap *map) {
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
 }

@@ -278,8 +278,7 @@ __global__ void __launch_bounds__(kGmThreads, 1)
                 words[4 * c + 2] = v.z;
                 words[4 * c + 3] = v.w;
             }
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&S.code_empty[cs]);
+            release_to_tma(&S.code_empty[cs], lane);
 #pragma unroll
             for (int gg = 0; gg < GPS; ++gg) {
                 if (gl >= GL) break;

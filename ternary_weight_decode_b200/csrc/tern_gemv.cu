@@ -290,12 +290,11 @@ __global__ void __launch_bounds__(kThreads)
         else
             process_d2<MT, NMAT, MODE>(stg, it, lane, row, act, KS, sq, L.GS, sc, L.sc_stride, yacc,
                                        p, n, (sb0 + it) * GPS);
+        // every lane's reads of the stage ordered before its TMA refill
+        fence_proxy_async_smem();
         __syncwarp();
         if (it + S < nsb) {
-            if (lane == 0) {
-                fence_proxy_async_smem();
-                issue(it + S);
-            }
+            if (lane == 0) issue(it + S);
             ++issued;
         }
     }

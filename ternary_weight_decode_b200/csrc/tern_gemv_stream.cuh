@@ -717,21 +717,18 @@ __global__ void __launch_bounds__(kSkThreads, 1)
                     // handed back when the item is done.
                     sk_item<FMT, MT>([&](int cc) { return lds128(wt + ((cc ^ rsw) << 4)); }, sc,
                                      act + sb * POS, L.Kpad, sq + sb * GPS * 4, L.GT, yacc, sink);
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive(&empty[kcs]);
+                    release_to_tma(&empty[kcs], lane);
                 } else {
                     // copied to registers, the slot handed back at once
                     uint4 wv[8];
 #pragma unroll
                     for (int cc = 0; cc < 8; ++cc) wv[cc] = lds128(wt + ((cc ^ rsw) << 4));
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive(&empty[kcs]);
+                    release_to_tma(&empty[kcs], lane);
                     sk_item<FMT, MT>([&](int cc) { return wv[cc]; }, sc, act + sb * POS, L.Kpad,
                                      sq + sb * GPS * 4, L.GT, yacc, sink);
                 }
             } else {
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&empty[kcs]);
+                release_to_tma(&empty[kcs], lane);
 #pragma unroll
                 for (int m = 0; m < MT; ++m) yacc[m] = 0.0f;
             }

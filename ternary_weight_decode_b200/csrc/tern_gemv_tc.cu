@@ -385,12 +385,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         process_superblock<FMT, MT, NMAT>(ctx, wstages + st * L.stage_bytes, lane, groups, it,
                                           corr_slot, yacc);
         groups += GPS;
+        // every lane's reads of the stage ordered before its TMA refill
+        fence_proxy_async_smem();
         __syncwarp();
         if (it + S < nsb) {
-            if (lane == 0) {
-                fence_proxy_async_smem();
-                issue(it + S);
-            }
+            if (lane == 0) issue(it + S);
             ++issued;
         }
     }

@@ -126,7 +126,8 @@ def test_verify_sizes_match_oracle(fmt, N, K, M):
 
 
 @pytest.mark.parametrize("fmt", FMTS)
-@pytest.mark.parametrize("K,N,M", [(5120, 17408, 64), (17408, 5120, 128), (17408, 5120, 24)])
+@pytest.mark.parametrize("K,N,M", [(5120, 17408, 64), (17408, 5120, 128), (17408, 5120, 24),
+                                   (5120, 17408, 4), (17408, 5120, 8)])
 def test_verify_full_shapes_sampled(fmt, K, N, M):
     """The 27B-shaped gate/up and down matrices at verify sizes, in the
     launch configuration the bench times, checked on sampled rows."""
