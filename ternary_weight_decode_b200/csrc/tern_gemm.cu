@@ -238,23 +238,42 @@ __global__ void __launch_bounds__(kGmThreads, 1)
     } else if (warp == 1) {
         // ------------------------------------------------------------- MMA
         if (lane == 0) {
+            // The issuing thread shares its scheduler with busy decode and
+            // epilogue warps, so its loop is kept short: stage indices and
+            // barrier parities advance incrementally, and the descriptors are
+            // a stage's base plus 2 per 32-byte K step (the start-address
+            // field counts 16-byte units and stays inside its 14 bits).
             const uint32_t idesc = idesc_i8(kGmTileN, TM, 1, 1);
+            const uint64_t a_desc0 = smem_desc_sw128(smem_u32(S.a[0]));
+            const uint64_t q_desc0 = smem_desc_sw128(smem_u32(S.act[0]));
+            constexpr uint64_t kAStep = kGmTile >> 4, kQStep = Sh::kActTile >> 4;
+            int as = 0, qs = 0, buf = 0;
+            uint32_t pa = 0, pq = 0, pe = 1;
             for (int gl = 0; gl < GL; ++gl) {
-                const int as = gl % kGmAStages, qs = gl % kGmActStages, buf = gl % kGmAccBufs;
-                bool ok = mbar_wait_bounded(&S.a_full[as], (gl / kGmAStages) & 1);
-                ok = ok && mbar_wait_bounded(&S.act_full[qs], (gl / kGmActStages) & 1);
-                if (gl >= kGmAccBufs)
-                    ok = ok && mbar_wait_bounded(&S.acc_empty[buf], ((gl / kGmAccBufs) - 1) & 1);
+                bool ok = mbar_wait_bounded(&S.a_full[as], pa);
+                ok = ok && mbar_wait_bounded(&S.act_full[qs], pq);
+                if (gl >= kGmAccBufs) ok = ok && mbar_wait_bounded(&S.acc_empty[buf], pe);
                 if (!ok) break;
                 tc_fence_after_sync();
-                const uint32_t a0 = smem_u32(S.a[as]), b0 = smem_u32(S.act[qs]);
+                const uint64_t ad = a_desc0 + as * kAStep, qd = q_desc0 + qs * kQStep;
+                const uint32_t d = tmem + buf * TM;
 #pragma unroll
-                for (int s = 0; s < 4; ++s)
-                    mma_i8_ss(tmem + buf * TM, smem_desc_sw128(a0 + 32 * s),
-                              smem_desc_sw128(b0 + 32 * s), idesc, s > 0);
+                for (int s = 0; s < 4; ++s) mma_i8_ss(d, ad + 2 * s, qd + 2 * s, idesc, s > 0);
                 tc_commit(&S.acc_full[buf]);
                 tc_commit(&S.a_empty[as]);
                 tc_commit(&S.act_empty[qs]);
+                if (++as == kGmAStages) {
+                    as = 0;
+                    pa ^= 1;
+                }
+                if (++qs == kGmActStages) {
+                    qs = 0;
+                    pq ^= 1;
+                }
+                if (++buf == kGmAccBufs) {
+                    buf = 0;
+                    pe ^= 1;
+                }
             }
         }
     } else if (warp < 2 + kGmDecodeWarps) {
