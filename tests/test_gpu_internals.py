@@ -137,3 +137,32 @@ def test_gemm_partials_bit_exact(fmt, M, N, K):
     ref = oracle.gemv(w, sw, q, s)
     assert np.max(np.abs(y.cpu().numpy() - ref)) <= tolerance(ref)
     assert tern.tern_device_error() == 0
+
+
+@pytest.mark.parametrize("fmt", [tern.TERN_FMT_2BIT, tern.TERN_FMT_BITPLANE])
+def test_streamed_partials_stable_under_ring_reuse(fmt):
+    """The 2-bit and bit-plane items hand their ring slot back as soon as the
+    codes are in registers, and the producer refills it by TMA at once.  A
+    missing proxy fence between the consumers' reads and that refill showed
+    as a few wrong partials in about one run of ten; thirty repeats of the
+    gate/up launch, every partial of both matrices bit for bit."""
+    N, K, M = 17408, 5120, 1
+    wg, wu = synth.trits(45, 0, N, K), synth.trits(45, 2, N, K)
+    G = synth.groups(K)
+    sg, su = synth.scales(45, 1, N, G), synth.scales(45, 3, N, G)
+    xh, x = _x(630, M, K)
+    q_ref, _ = oracle.act_quant(xh, fwht_block=128, rmsnorm=True)
+    Pg, Pu = oracle.group_partials(wg, q_ref), oracle.group_partials(wu, q_ref)
+    mats = [make_matrix(fmt, w, sw).retile_scales() for w, sw in ((wg, sg), (wu, su))]
+    h = torch.empty((M, N), dtype=torch.float32, device="cuda")
+    q = torch.empty((M, K), dtype=torch.int8, device="cuda")
+    s = torch.empty((M,), dtype=torch.float32, device="cuda")
+    P = torch.empty((2, M, N, G), dtype=torch.int32, device="cuda")
+    ws = tern.stream_workspace(fmt, N, M, True)
+    for rep in range(30):
+        P.fill_(-(1 << 30))
+        tern.tern_debug_streamed(mats[0], mats[1], x, h, q, s, P, ws, qflags=RMS | ROT, M=M)
+        torch.cuda.synchronize()
+        got = P.cpu().numpy()
+        assert np.array_equal(got[0], Pg) and np.array_equal(got[1], Pu), f"repeat {rep}"
+    assert tern.tern_device_error() == 0
