@@ -356,9 +356,17 @@ __global__ void __launch_bounds__(kGmThreads, 1)
                     __syncwarp();
                     if (lane == 0) mbar_arrive(&S.acc_empty[buf]);
                 }
+                // acc += s * float(P), two columns per packed FMA (each lane
+                // rounds as fmaf does)
 #pragma unroll
-                for (int c = 0; c < 8; ++c)
-                    acc[8 * h + c] = fmaf(s, __int2float_rn(static_cast<int>(v[c])), acc[8 * h + c]);
+                for (int c = 0; c < 8; c += 2) {
+                    const float2 a2 = __ffma2_rn(make_float2(s, s),
+                                                 make_float2(__int2float_rn(static_cast<int>(v[c])),
+                                                             __int2float_rn(static_cast<int>(v[c + 1]))),
+                                                 make_float2(acc[8 * h + c], acc[8 * h + c + 1]));
+                    acc[8 * h + c] = a2.x;
+                    acc[8 * h + c + 1] = a2.y;
+                }
                 if constexpr (DBG) {
                     // test hook: the exact partials of this group
 #pragma unroll
