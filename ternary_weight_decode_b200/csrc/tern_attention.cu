@@ -413,13 +413,18 @@ int split_ctas_per_sm(int GQ) {
 }  // namespace
 
 int attention_chunk(int L, int Hkv, int GQ, int num_sms) {
-    // Chunks of whole passes, chosen so that the CTAs fill whole waves of
-    // the SMs: the least tokens that one resident CTA slot has to stream
-    // (waves x chunk), the fewer CTAs on a tie.
+    // Chunks of at least one pass, beyond that of whole warps' worth of
+    // tokens (the last pass may be partial), chosen so that the CTAs fill
+    // whole waves of the SMs: the least tokens that one resident CTA slot has
+    // to stream (waves x chunk), the fewer CTAs on a tie.  (Chunks shorter
+    // than a pass measured slower: a CTA's fixed work and the merge grow.)
     // At most kAttMaxChunks chunks (the merge keeps one weight per chunk in
     // shared memory).
     const long long slots = static_cast<long long>(split_ctas_per_sm(GQ)) * num_sms;
-    auto whole_passes = [](long long t) { return (t + kAttThreads - 1) / kAttThreads * kAttThreads; };
+    constexpr long long kGrain = 32;
+    auto whole_passes = [](long long t) {
+        return t <= kAttThreads ? static_cast<long long>(kAttThreads) : (t + kGrain - 1) / kGrain * kGrain;
+    };
     long long best = whole_passes((L + kAttMaxChunks - 1) / kAttMaxChunks), best_cost = -1;
     for (long long w = 1; w <= 64; ++w) {
         const long long per_head = w * slots / Hkv > 0 ? w * slots / Hkv : 1;
