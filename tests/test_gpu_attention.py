@@ -49,7 +49,10 @@ def test_append_matches_oracle_q4_0_bit_for_bit():
 
 @pytest.mark.parametrize("Hq,Hkv,L", [(40, 8, 1), (40, 8, 7), (40, 8, 128), (40, 8, 129), (40, 8, 1000),
                                       (40, 8, 4097), (8, 8, 300), (16, 8, 513), (32, 8, 2048),
-                                      (8, 1, 5000), (10, 2, 33)])
+                                      (8, 1, 5000), (10, 2, 33),
+                                      # chunks longer than one pass of 128 and ending in a partial
+                                      # pass (160 and 288 tokens on 148 SMs), and a short last chunk
+                                      (40, 8, 10000), (40, 8, 20001)])
 def test_attention_matches_oracle(Hq, Hkv, L):
     rng = np.random.default_rng(Hq * 1000 + L)
     k, v = _kv(rng, Hkv, L, 0.3)
