@@ -332,11 +332,12 @@ __global__ void __launch_bounds__(kSkThreads, 1)
                        const __grid_constant__ CUtensorMap tm3_1, const SkParams p) {
     constexpr int NMAT = (MODE == kModeSwiglu) ? 2 : 1;
     constexpr int CH = kSkChunk / NMAT;  // units of one matrix per ring chunk
-    // Base-3 with one token row rotates every slot of a round (see pass 1):
-    // rounds of 3 (one round up to K = 6144) waste fewer rotations on empty
-    // slots than rounds of 5, at the price of a second round for the down
-    // projection (measured: base-3 step -0.8 %).
-    constexpr int KEEP = (MT == 1 && FMT == TERN_FMT_BASE3) ? 3 : kSkKeep;
+    // Base-3 with one token row processes every slot of a round (see pass 1):
+    // the rotated gate/up input takes rounds of 3 (one round up to K = 6144),
+    // which waste fewer rotations on empty slots than rounds of 5 (gate/up
+    // 16.2 -> 15.7 us); the unrotated projections keep rounds of 5, which
+    // spare the down projection (K = 17408) a second round (12.3 vs 13.1 us).
+    constexpr int KEEP = (MT == 1 && FMT == TERN_FMT_BASE3 && MODE == kModeSwiglu) ? 3 : kSkKeep;
     constexpr int POS = Fmt<FMT>::kPos;
     constexpr int GPS = Fmt<FMT>::kGroups;
     constexpr int SCB = scb<FMT>();
