@@ -11,17 +11,20 @@ with the decode-step rate (tok/s-equivalent) beside it.
 
 The same JSON line carries the other workloads under "configs":
   c1  single GEMV K = N = 256, M = 1 (microseconds per call);
-  c2  one 27B-shaped layer, base-3 and 2-bit, rotating 8 independent layers
-      so the weights never sit in L2, with the per-projection split;
-  c3_2bit  the 64-layer step in the 2-bit format;
-  c4  gate/up + SwiGLU and down at M = 1, 2, 4, 8, 16 token rows (GB/s, TOPS);
-  c5  prefill GEMM, (K, N) = (5120, 17408) and (17408, 5120), M = 512 / 2048 / 8192;
+  c2  one 27B-shaped layer, base-3, 2-bit and bit-plane, rotating 8
+      independent layers so the weights never sit in L2, with the
+      per-projection split;
+  c3_2bit, c3_bitplane  the 64-layer step in the other two formats;
+  c4  gate/up + SwiGLU and down at M = 1, 2, 4, 8, 16 token rows (GB/s, TOPS),
+      each format;
+  c5  prefill GEMM, (K, N) = (5120, 17408) and (17408, 5120), M = 512 / 2048 / 8192,
+      each format;
   c6  multi-token verify: the gate and down GEMMs at M = 16 .. 128 on the tensor cores;
   c7  decode attention over a Q4_0 KV cache at 4K / 16K / 64K tokens;
 each with a bounded sample of the CPU oracle timed on this host.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--fmt base3|2bit] [--layers 64] [--M 1] [--quick]
+                    [--fmt base3|2bit|bitplane] [--layers 64] [--M 1] [--quick]
     python bench.py --attention 4096 65536      # c7 alone
 
 N > 1 runs N independent replicas (one process per GPU, launched by
@@ -707,8 +710,7 @@ def other_format(name, x0, steps, peak, stream):
                           "frac": ob / (oms * 1e-3) / 1e9 / peak, "tok_s_equiv": 1e3 / oms,
                           "bytes_per_step": ob},
            "c2_" + name: layer_configs(om, fmt, peak)}
-    if fmt != 2:
-        out["c4_" + name] = ffn_sweep(om, fmt, peak)
+    out["c4_" + name] = ffn_sweep(om, fmt, peak)
     del om
     return out
 
@@ -838,7 +840,7 @@ def main():
                 configs.update(other_format(other, x0, args.steps, peak, stream))
                 torch.cuda.empty_cache()
         if not args.no_prefill:
-            configs["c5"] = [prefill_gemm(f, K, N) for f in (0, 1)
+            configs["c5"] = [prefill_gemm(f, K, N) for f in (0, 1, 2)
                              for K, N in ((HIDDEN, FFN), (FFN, HIDDEN))]
         configs["c7_attention"] = attention_sweep()
         if not args.no_cpu_baseline:

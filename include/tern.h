@@ -52,9 +52,9 @@ typedef enum {
     TERN_FMT_BASE3 = 0,   /* 5 trits per byte (PTQ1_0-style), 1.6 bit/trit */
     TERN_FMT_2BIT = 1,    /* 4 trits per byte (PQ2-style), 2 bit/trit */
     TERN_FMT_BITPLANE = 2 /* a nonzero bit and a sign bit per weight, 2 bit/trit (Bonsai
-                             page, "后面还有没有优化空间"); the format calls and the
-                             streamed entry points take it, the other compute calls
-                             return TERN_EUNSUPPORTED */
+                             page, "后面还有没有优化空间"); every call takes it except
+                             the tensor-core GEMV engine of tern_debug_select_engine,
+                             which returns TERN_EUNSUPPORTED for it */
 } tern_format;
 
 /* Bit 0 of tern_matrix.flags: the packed codes and scales are not written by
@@ -519,8 +519,10 @@ tern_status tern_debug_mma_i8(int32_t a_in_smem, const int8_t *A, int32_t a_sign
 /*
  * Test hook: selects the engine of the GEMV entry points for the calling
  * process -- 0: tensor cores (tcgen05), 1: CUDA cores (dp4a, the default).
- * Both compute the same integers; the tests compare them.
- * tern_debug_group_partials always uses the CUDA-core engine.
+ * Both compute the same integers; the tests compare them.  The tensor-core
+ * engine has no bit-plane form: with it selected, a bit-plane matrix gives
+ * TERN_EUNSUPPORTED.  tern_debug_group_partials always uses the CUDA-core
+ * engine.
  */
 tern_status tern_debug_select_engine(int32_t engine);
 

@@ -253,8 +253,6 @@ tern_status act_quant_fwht(const void *x, int32_t x_is_fp16, int32_t M, int32_t 
 }
 
 static tern_status run_gemv(tern::GemvLaunch &L, const char *name, cudaStream_t s) {
-    if (L.fmt == TERN_FMT_BITPLANE)
-        return fail(TERN_EUNSUPPORTED, "%s: the bit-plane format runs on the streamed entry points only", name);
     const char *why = nullptr;
     cudaError_t e = tern::launch_gemv(L, s, &why);
     if (why) return fail(TERN_EUNSUPPORTED, "%s", why);
@@ -518,8 +516,6 @@ static tern_status run_gemm(const tern_matrix *W, const int8_t *q, int32_t ldq, 
                             int32_t M, float *y, int32_t ldy, int32_t *dbg_P, void *stream) {
     tern_status st = check_matrix(W, "tern_gemm");
     if (st != TERN_OK) return st;
-    if (W->fmt == TERN_FMT_BITPLANE)
-        return fail(TERN_EUNSUPPORTED, "tern_gemm: the bit-plane format runs on the streamed entry points only%s");
     if (M < 1) return fail(TERN_EINVAL, "tern_gemm: M must be >= 1%s");
     if (!q || !aligned(q, 16) || ldq < W->K || ldq % 16 != 0)
         return fail(TERN_EINVAL, "tern_gemm: q must be 16-byte aligned with ldq >= K, ldq %% 16 == 0%s");

@@ -19,7 +19,8 @@
 //    the tensor cores run one group ahead of the epilogue;
 //  * warps 2..5 (decode; a thread = one weight row): the row's 32 code words
 //    of the superblock into registers, then per group the signed int8
-//    weights w = t - 1 into a 128 x 128 B tile in the 128-byte-swizzled
+//    weights (w = t - 1 for D3 and D2; from the two bit planes for DB)
+//    into a 128 x 128 B tile in the 128-byte-swizzled
 //    K-major layout the MMA reads (trits never leave the SM), two tiles in
 //    flight;
 //  * warps 6..21 (epilogue, four per tensor-memory lane quarter, 64 token
@@ -118,6 +119,19 @@ __device__ __forceinline__ void decode_half(const uint32_t (&words)[32], int gg,
                 const int d = 5 * cw + i - d0;
                 if (d >= 0 && d < 16) wq[d] = signed_trits(t[i]);
             }
+        }
+    } else if constexpr (FMT == TERN_FMT_BITPLANE) {
+        // DB: word pair p (nonzero plane n, sign plane s) holds positions
+        // 32p + 4i + j in bit 8j + i; group gg = pairs 4gg .. 4gg+3.  With
+        // a = the n bits and b = the (n AND s) bits of four positions (one
+        // per byte), w = a + 0xFE b is 0x01, 0xFF or 0 per byte: no carries.
+#pragma unroll
+        for (int pr = 0; pr < 2; ++pr) {
+            const uint32_t nz = words[8 * gg + 4 * H + 2 * pr];
+            const uint32_t ng = nz & words[8 * gg + 4 * H + 2 * pr + 1];
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+                wq[8 * pr + i] = ((nz >> i) & 0x01010101u) + 0xFEu * ((ng >> i) & 0x01010101u);
         }
     } else {
         // D2: code word w holds positions 16w + 4i + j in bits [2i, 2i+1] of
@@ -449,10 +463,12 @@ cudaError_t launch_gemm_tm(const GemmLaunch &L, const GemmParams &p, int C, cuda
         *why = "K too large for the shared-memory scale block of the prefill GEMM (K <= 40960)";
         return cudaErrorInvalidValue;
     }
-    auto kern = L.dbg_P ? (L.fmt == TERN_FMT_BASE3 ? gemm_kernel<TERN_FMT_BASE3, true, TM>
-                                                   : gemm_kernel<TERN_FMT_2BIT, true, TM>)
-                        : (L.fmt == TERN_FMT_BASE3 ? gemm_kernel<TERN_FMT_BASE3, false, TM>
-                                                   : gemm_kernel<TERN_FMT_2BIT, false, TM>);
+    auto kern = L.dbg_P ? (L.fmt == TERN_FMT_BASE3      ? gemm_kernel<TERN_FMT_BASE3, true, TM>
+                           : L.fmt == TERN_FMT_BITPLANE ? gemm_kernel<TERN_FMT_BITPLANE, true, TM>
+                                                        : gemm_kernel<TERN_FMT_2BIT, true, TM>)
+                        : (L.fmt == TERN_FMT_BASE3      ? gemm_kernel<TERN_FMT_BASE3, false, TM>
+                           : L.fmt == TERN_FMT_BITPLANE ? gemm_kernel<TERN_FMT_BITPLANE, false, TM>
+                                                        : gemm_kernel<TERN_FMT_2BIT, false, TM>);
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(smem));
     if (e != cudaSuccess) return e;

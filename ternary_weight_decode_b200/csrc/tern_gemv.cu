@@ -10,7 +10,10 @@
 //
 // This engine decodes a D3 word into five int8x4 digit words t_i = D_i -
 // 3 D_(i-1) and dots them with dp4a (sum w q = sum t q - sum q per group);
-// D2 fields are (X >> 2i) & 0x03030303.  Each warp streams its own
+// D2 fields are (X >> 2i) & 0x03030303.  A DB (bit-plane) pair is dotted
+// plane by plane, the nonzero plane and the negative one (nonzero AND sign)
+// masked one bit per byte (sum w q = sum n q - 2 sum (n s) q, nothing to
+// subtract per group).  Each warp streams its own
 // superblocks through a ring of TMA stages (32 x 128 B box per matrix,
 // 128-byte swizzle, L2 evict-first, no multicast).  This is the default
 // engine; the tensor-core engine (tern_gemv_tc.cu) replaces the dp4a with
@@ -55,12 +58,14 @@ __host__ __device__ inline CcLayout cc_layout(int sb_per_cta, int stages) {
 }
 
 // Adds one finished group to the fp32 accumulators (or stores its partials).
-template <int MT, int NMAT, int MODE>
+// SUBQ: the accumulators hold sum t q with t = w + 1 (D3, D2), so the group
+// sum of q is subtracted; a DB accumulator already holds sum w q.
+template <int MT, int NMAT, int MODE, bool SUBQ = true>
 __device__ __forceinline__ void finish_group(int (&acc)[NMAT][MT], float (&yacc)[NMAT][MT], int m,
                                              int gl, int row, const int *sq, int GS,
                                              const float *sc, int sc_stride,
                                              const GemvParams &p, int n, int gg) {
-    const int s = sq[m * GS + gl];
+    const int s = SUBQ ? sq[m * GS + gl] : 0;
 #pragma unroll
     for (int mat = 0; mat < NMAT; ++mat) {
         const int P = acc[mat][m] - s;
@@ -197,6 +202,87 @@ __device__ __forceinline__ void process_d2(const uint8_t *stage, int sbl, int la
     }
 }
 
+// DB: each 16-byte chunk holds two word pairs (nonzero plane n, sign plane
+// s) of 32 positions; bit 8j + i of a word is position 4i + j of its pair,
+// so the byte mask 0x01010101 << i lines the pair's bits up with activation
+// word i of the pair.
+template <int MT, int NMAT, int MODE>
+__device__ __forceinline__ void process_db(const uint8_t *stage, int sbl, int lane, int row,
+                                           const uint8_t *act, int KS, const int *sq, int GS,
+                                           const float *sc, int sc_stride,
+                                           float (&yacc)[NMAT][MT], const GemvParams &p, int n,
+                                           int g_base) {
+    int acc[NMAT][MT];
+#pragma unroll
+    for (int mat = 0; mat < NMAT; ++mat)
+#pragma unroll
+        for (int m = 0; m < MT; ++m) acc[mat][m] = 0;
+    const int rsw = lane & 7;
+    const int gl0 = sbl * 4;
+#pragma unroll
+    for (int c = 0; c < 8; ++c) {
+        uint32_t words[NMAT][4];
+#pragma unroll
+        for (int mat = 0; mat < NMAT; ++mat) {
+            uint4 wv = lds128(stage + mat * kTile + lane * kSBBytes + ((c ^ rsw) << 4));
+            words[mat][0] = wv.x;
+            words[mat][1] = wv.y;
+            words[mat][2] = wv.z;
+            words[mat][3] = wv.w;
+        }
+#pragma unroll
+        for (int m = 0; m < MT; ++m) {
+            const uint8_t *a = act + m * KS + sbl * 512 + c * 64;
+            uint32_t aw[16];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                uint4 v = lds128(a + 16 * j);
+                aw[4 * j + 0] = v.x;
+                aw[4 * j + 1] = v.y;
+                aw[4 * j + 2] = v.z;
+                aw[4 * j + 3] = v.w;
+            }
+#pragma unroll
+            for (int mat = 0; mat < NMAT; ++mat) {
+                int sn = 0, sg = 0;
+                if (MT <= 2) {
+                    // masked bits: lane values 2^i * bit, summed per i and
+                    // rescaled (exactly) by arithmetic shifts
+                    int an[8] = {0, 0, 0, 0, 0, 0, 0, 0}, as[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+#pragma unroll
+                    for (int pr = 0; pr < 2; ++pr) {
+                        const uint32_t nz = words[mat][2 * pr], ng = nz & words[mat][2 * pr + 1];
+#pragma unroll
+                        for (int i = 0; i < 8; ++i) {
+                            an[i] = dp4a_us(nz & (0x01010101u << i), aw[8 * pr + i], an[i]);
+                            as[i] = dp4a_us(ng & (0x01010101u << i), aw[8 * pr + i], as[i]);
+                        }
+                    }
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) {
+                        sn += an[i] >> i;
+                        sg += as[i] >> i;
+                    }
+                } else {
+#pragma unroll
+                    for (int pr = 0; pr < 2; ++pr) {
+                        const uint32_t nz = words[mat][2 * pr], ng = nz & words[mat][2 * pr + 1];
+#pragma unroll
+                        for (int i = 0; i < 8; ++i) {
+                            sn = dp4a_us((nz >> i) & 0x01010101u, aw[8 * pr + i], sn);
+                            sg = dp4a_us((ng >> i) & 0x01010101u, aw[8 * pr + i], sg);
+                        }
+                    }
+                }
+                acc[mat][m] += sn - 2 * sg;
+            }
+            if (c & 1)
+                finish_group<MT, NMAT, MODE, false>(acc, yacc, m, gl0 + (c >> 1), row, sq, GS, sc,
+                                                    sc_stride, p, n, g_base + (c >> 1));
+        }
+    }
+}
+
 template <int FMT, int MT, int MODE, int XIN>
 __global__ void __launch_bounds__(kThreads)
     gemv_cc_kernel(const __grid_constant__ CUtensorMap tm0, const __grid_constant__ CUtensorMap tm1,
@@ -286,6 +372,9 @@ __global__ void __launch_bounds__(kThreads)
         const uint8_t *stg = wstages + st * L.stage_bytes;
         if (FMT == TERN_FMT_BASE3)
             process_d3<MT, NMAT, MODE>(stg, it, lane, row, act, KS, sq, L.GS, sc, L.sc_stride, yacc,
+                                       p, n, (sb0 + it) * GPS);
+        else if (FMT == TERN_FMT_BITPLANE)
+            process_db<MT, NMAT, MODE>(stg, it, lane, row, act, KS, sq, L.GS, sc, L.sc_stride, yacc,
                                        p, n, (sb0 + it) * GPS);
         else
             process_d2<MT, NMAT, MODE>(stg, it, lane, row, act, KS, sq, L.GS, sc, L.sc_stride, yacc,
@@ -526,8 +615,15 @@ void fill_params(GemvParams &p, const GemvLaunch &L) {
 void select_engine(int engine) { g_engine = engine; }
 
 cudaError_t launch_gemv(const GemvLaunch &L, cudaStream_t s, const char **why) {
-    if (g_engine == 0 && L.mode != kModePartials) return launch_gemv_tc(L, s, why);
+    if (g_engine == 0 && L.mode != kModePartials) {
+        if (L.fmt == TERN_FMT_BITPLANE) {
+            *why = "the tensor-core GEMV engine has no bit-plane form";
+            return cudaErrorInvalidValue;
+        }
+        return launch_gemv_tc(L, s, why);
+    }
     if (L.fmt == TERN_FMT_BASE3) return launch_cc_fmt<TERN_FMT_BASE3>(L, s, why);
+    if (L.fmt == TERN_FMT_BITPLANE) return launch_cc_fmt<TERN_FMT_BITPLANE>(L, s, why);
     return launch_cc_fmt<TERN_FMT_2BIT>(L, s, why);
 }
 

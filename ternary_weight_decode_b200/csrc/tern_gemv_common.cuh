@@ -35,7 +35,7 @@ struct Fmt<TERN_FMT_2BIT> {
     static constexpr int kGroups = 4;
 };
 template <>
-struct Fmt<TERN_FMT_BITPLANE> {  // the streamed kernels only
+struct Fmt<TERN_FMT_BITPLANE> {  // every engine but the tensor-core GEMV
     static constexpr int kPos = 512;
     static constexpr int kGroups = 4;
 };

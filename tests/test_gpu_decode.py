@@ -64,7 +64,7 @@ def check_layer(rec, l, rng, nrows=48):
         assert np.max(np.abs(x_after_down[:, r] - ref)) <= tolerance(ref)
 
 
-@pytest.mark.parametrize("fmt", [tern.TERN_FMT_BASE3, tern.TERN_FMT_2BIT])
+@pytest.mark.parametrize("fmt", [tern.TERN_FMT_BASE3, tern.TERN_FMT_2BIT, tern.TERN_FMT_BITPLANE])
 @pytest.mark.parametrize("mode", ["streamed", "fused"])
 def test_decode_step_64_layers_sampled(fmt, mode):
     model = decode.DecodeModel(fmt, 64, M=1, mode=mode).build(seed_base=0)
@@ -81,10 +81,11 @@ def test_decode_step_64_layers_sampled(fmt, mode):
     assert tern.tern_device_error() == 0
 
 
+@pytest.mark.parametrize("fmt", [tern.TERN_FMT_BASE3, tern.TERN_FMT_BITPLANE])
 @pytest.mark.parametrize("M", [2, 4, 16])
-def test_decode_layers_multi_slot(M):
+def test_decode_layers_multi_slot(fmt, M):
     mode = "streamed" if M <= 2 else "fused"
-    model = decode.DecodeModel(tern.TERN_FMT_BASE3, 2, M=M, mode=mode).build(seed_base=0)
+    model = decode.DecodeModel(fmt, 2, M=M, mode=mode).build(seed_base=0)
     x0 = synth.activation_rows([1000 + r for r in range(M)], H).astype(np.float32)
     model.x.copy_(torch.from_numpy(x0))
     rec = []

@@ -115,16 +115,21 @@ def test_bitplane_invalid_bits_are_counted():
     assert int(bad.item()) == 1
 
 
-def test_bitplane_rejected_by_the_non_streamed_kernels():
+def test_bitplane_rejected_only_by_the_tensor_core_gemv_engine():
     N, K = 64, 256
     w = synth.trits(13, 0, N, K)
     M = make_matrix(tern.TERN_FMT_BITPLANE, w, synth.scales(13, 1, N, 2))
     q = torch.zeros((1, K), dtype=torch.int8, device="cuda")
     s = torch.ones(1, dtype=torch.float32, device="cuda")
     y = torch.zeros((1, N), dtype=torch.float32, device="cuda")
-    with pytest.raises(tern.TernError) as e:
-        tern.tern_gemv(M, q, s, y)
-    assert e.value.status == tern.TERN_EUNSUPPORTED
-    with pytest.raises(tern.TernError) as e:
-        tern.tern_gemm(M, q, s, y)
-    assert e.value.status == tern.TERN_EUNSUPPORTED
+    tern.tern_debug_select_engine(tern.ENGINE_TENSOR_CORES)
+    try:
+        with pytest.raises(tern.TernError) as e:
+            tern.tern_gemv(M, q, s, y)
+        assert e.value.status == tern.TERN_EUNSUPPORTED
+    finally:
+        tern.tern_debug_select_engine(tern.ENGINE_CUDA_CORES)
+    tern.tern_gemv(M, q, s, y)   # the CUDA-core engine and the GEMM take it
+    tern.tern_gemm(M, q, s, y)
+    torch.cuda.synchronize()
+    assert not y.any()

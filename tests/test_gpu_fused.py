@@ -10,7 +10,7 @@ from ternary_weight_decode_b200 import synth, tern
 from gpu_util import make_matrix, to_dev, tolerance
 
 pytestmark = pytest.mark.gpu
-FMTS = [tern.TERN_FMT_BASE3, tern.TERN_FMT_2BIT]
+FMTS = [tern.TERN_FMT_BASE3, tern.TERN_FMT_2BIT, tern.TERN_FMT_BITPLANE]
 RMS, ROT = tern.TERN_QUANT_RMSNORM, tern.TERN_QUANT_FWHT128
 
 

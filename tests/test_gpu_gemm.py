@@ -12,7 +12,7 @@ from ternary_weight_decode_b200 import synth, tern
 from gpu_util import make_matrix, padded_q, to_dev, tolerance
 
 pytestmark = pytest.mark.gpu
-FMTS = [tern.TERN_FMT_BASE3, tern.TERN_FMT_2BIT]
+FMTS = [tern.TERN_FMT_BASE3, tern.TERN_FMT_2BIT, tern.TERN_FMT_BITPLANE]
 
 
 def quantised(seed, M, K):
@@ -68,6 +68,7 @@ def big_matrix(fmt, N, K, seed):
 @pytest.mark.parametrize("fmt,K,N,M", [(tern.TERN_FMT_BASE3, 5120, 17408, 512),
                                        (tern.TERN_FMT_BASE3, 17408, 5120, 512),
                                        (tern.TERN_FMT_2BIT, 5120, 17408, 2048),
+                                       (tern.TERN_FMT_BITPLANE, 17408, 5120, 2048),
                                        (tern.TERN_FMT_BASE3, 5120, 17408, 8192)])
 def test_gemm_prefill_shapes_sampled(fmt, K, N, M):
     seed = 40 + M

@@ -12,7 +12,7 @@ from gpu_util import make_matrix, padded_q, to_dev, tolerance
 
 pytestmark = pytest.mark.gpu
 
-FMTS = [tern.TERN_FMT_BASE3, tern.TERN_FMT_2BIT]
+FMTS = [tern.TERN_FMT_BASE3, tern.TERN_FMT_2BIT, tern.TERN_FMT_BITPLANE]
 SHAPES = [(256, 256), (37, 300), (100, 1280), (33, 5120), (64, 641), (5, 17408), (1, 1), (32, 20)]
 
 

@@ -115,7 +115,7 @@ def test_streamed_codes_equal_act_quant_entry_point(fmt, K, qflags):
         np.testing.assert_array_equal(s, sa.cpu().numpy())
 
 
-@pytest.mark.parametrize("fmt", FMTS[:2])
+@pytest.mark.parametrize("fmt", FMTS)
 @pytest.mark.parametrize("M,N,K", [(300, 200, 1000), (256, 512, 17408), (17, 130, 5120)])
 def test_gemm_partials_bit_exact(fmt, M, N, K):
     """The tensor-core accumulator of the prefill GEMM holds the exact group
