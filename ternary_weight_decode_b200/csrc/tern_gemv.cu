@@ -161,6 +161,17 @@ __device__ __forceinline__ void process_d2(const uint8_t *stage, int sbl, int la
             words[mat][2] = wv.z;
             words[mat][3] = wv.w;
         }
+        // several token rows: the digit words once per chunk, shared by
+        // every row (as the D3 path does)
+        uint32_t t[NMAT][16];
+        if (MT > 2) {
+#pragma unroll
+            for (int mat = 0; mat < NMAT; ++mat)
+#pragma unroll
+                for (int wi = 0; wi < 4; ++wi)
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) t[mat][4 * wi + i] = (words[mat][wi] >> (2 * i)) & 0x03030303u;
+        }
 #pragma unroll
         for (int m = 0; m < MT; ++m) {
             const uint8_t *a = act + m * KS + sbl * 512 + c * 64;
@@ -188,11 +199,7 @@ __device__ __forceinline__ void process_d2(const uint8_t *stage, int sbl, int la
                     acc[mat][m] += a4[0] + (a4[1] >> 2) + (a4[2] >> 4) + (a4[3] >> 6);
                 } else {
 #pragma unroll
-                    for (int wi = 0; wi < 4; ++wi)
-#pragma unroll
-                        for (int i = 0; i < 4; ++i)
-                            acc[mat][m] = dp4a_ss((words[mat][wi] >> (2 * i)) & 0x03030303u,
-                                                  aw[4 * wi + i], acc[mat][m]);
+                    for (int d = 0; d < 16; ++d) acc[mat][m] = dp4a_ss(t[mat][d], aw[d], acc[mat][m]);
                 }
             }
             if (c & 1)
@@ -230,6 +237,20 @@ __device__ __forceinline__ void process_db(const uint8_t *stage, int sbl, int la
             words[mat][2] = wv.z;
             words[mat][3] = wv.w;
         }
+        // several token rows: signed weight words once per chunk (a + 0xFE b
+        // per byte: 1, -1 or 0, no carries), shared by every row
+        uint32_t wq[NMAT][16];
+        if (MT > 2) {
+#pragma unroll
+            for (int mat = 0; mat < NMAT; ++mat)
+#pragma unroll
+                for (int pr = 0; pr < 2; ++pr) {
+                    const uint32_t nz = words[mat][2 * pr], ng = nz & words[mat][2 * pr + 1];
+#pragma unroll
+                    for (int i = 0; i < 8; ++i)
+                        wq[mat][8 * pr + i] = ((nz >> i) & 0x01010101u) + 0xFEu * ((ng >> i) & 0x01010101u);
+                }
+        }
 #pragma unroll
         for (int m = 0; m < MT; ++m) {
             const uint8_t *a = act + m * KS + sbl * 512 + c * 64;
@@ -263,18 +284,11 @@ __device__ __forceinline__ void process_db(const uint8_t *stage, int sbl, int la
                         sn += an[i] >> i;
                         sg += as[i] >> i;
                     }
+                    acc[mat][m] += sn - 2 * sg;
                 } else {
 #pragma unroll
-                    for (int pr = 0; pr < 2; ++pr) {
-                        const uint32_t nz = words[mat][2 * pr], ng = nz & words[mat][2 * pr + 1];
-#pragma unroll
-                        for (int i = 0; i < 8; ++i) {
-                            sn = dp4a_us((nz >> i) & 0x01010101u, aw[8 * pr + i], sn);
-                            sg = dp4a_us((ng >> i) & 0x01010101u, aw[8 * pr + i], sg);
-                        }
-                    }
+                    for (int d = 0; d < 16; ++d) acc[mat][m] = dp4a_ss(wq[mat][d], aw[d], acc[mat][m]);
                 }
-                acc[mat][m] += sn - 2 * sg;
             }
             if (c & 1)
                 finish_group<MT, NMAT, MODE, false>(acc, yacc, m, gl0 + (c >> 1), row, sq, GS, sc,
