@@ -480,6 +480,7 @@ cudaError_t launch_cc(const GemvLaunch &Lh, cudaStream_t s, const char **why) {
     if (want > 8) want = 8;
     if (nsplit < want) nsplit = want;
     if (nsplit > p.SB) nsplit = p.SB;
+    nsplit = even_split(p.SB, nsplit);
     p.sb_per_cta = static_cast<int>(ceil_div(p.SB, nsplit));
     p.nsplit = static_cast<int>(ceil_div(p.SB, p.sb_per_cta));
     if (MODE != kModePartials && p.nsplit > 8) {

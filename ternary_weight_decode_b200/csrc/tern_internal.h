@@ -15,6 +15,17 @@ namespace tern {
 
 inline int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
 
+// K split of the fused GEMV engines: nsplit, or the next count up to 8 (a
+// portable cluster) that divides the SB superblocks evenly, so that the
+// ranks of a cluster finish together (2-bit gate/up at K = 5120: 10
+// superblocks as 5 x 2, not 3 + 3 + 3 + 1).  Both engines take the same
+// split, hence the same sum order.
+inline int even_split(int SB, int nsplit) {
+    for (int n = nsplit; SB % nsplit != 0 && n <= 8 && n <= SB; ++n)
+        if (SB % n == 0) nsplit = n;
+    return nsplit;
+}
+
 // One-time set-up of a launch site on each device (kernel attributes, launch
 // plans).  Safe when several host threads make their first call at once: the
 // first caller on a device runs `setup` under a lock, later callers see its
